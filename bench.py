@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the Sparse VideoGen sparse-attention layer on B200.
+
+One step = the whole hot path on one synthetic layer resident in HBM:
+online profiling (+ its finalize kernel), block-mask construction for both
+patterns, permutation of Q/K/V for temporal heads, block-sparse attention and
+the inverse permutation of the temporal outputs.
+
+Prints ONE JSON line (rank 0). `value` is TFLOP/s counted on computed blocks
+(4*d per attended (query, key) pair, all heads, all ranks) divided by the
+measured step time; `roofline` reports the attention kernel alone. The dense
+baseline is the same attention kernel over the all-blocks mask.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import svg_inputs as SI  # noqa: E402
+
+METRIC = "sparse-attn layer ms & TFLOPS (computed blocks) vs BF16 peak; speedup vs dense"
+UNIT = "TFLOP/s (computed blocks)"
+DEFAULT_WORKLOAD = SI.HUNYUAN.name
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            pk = json.load(fh)
+        return {"bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                "hbm_gbs": pk["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "source": "fallback"}
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+def computed_pairs(svg, g, kind) -> int:
+    """(query, key) token pairs inside the computed blocks of one head."""
+    from video_dit_spatial_b200.layer import BlockMaskCSR
+    m = BlockMaskCSR(g, kind, "cuda")
+    m.build(g)
+    rp = m.row_ptr.cpu().numpy().astype(np.int64)
+    ci = m.col_idx.cpu().numpy()[:m.nnz].astype(np.int64)
+    N = g.N
+    rows_in = np.minimum(g.block_q, N - np.arange(g.n_qblocks) * g.block_q)
+    cols_in = np.minimum(g.block_k, N - np.arange(g.n_kblocks) * g.block_k)
+    counts = np.diff(rp)
+    return int(np.sum(np.repeat(rows_in, counts) * cols_in[ci]))
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", ident], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, flag in zip(names, parts[5:9]):
+                    if flag.lower().startswith("active"):
+                        reasons.add(n)
+            os.unlink(self.path)
+        except Exception:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline, and the --impl reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(wl, n_rows: int, heads, seed: int = 5):
+    """Times the fp64 oracle's layer output on n_rows query rows of `heads`.
+
+    Returns (seconds, flops) with flops = 4*d*attended keys of those rows.
+    """
+    import oracle as O
+    kinds = SI.planted_head_kinds(wl)
+    rng = np.random.default_rng(seed)
+    flops = 0
+    elapsed = 0.0
+    for h in heads:
+        q, k, v = (O.from_bf16_bits(t.view(torch.int16).numpy()) for t in SI.make_head(wl, 0, h))
+        rows = np.sort(rng.choice(wl.N, size=n_rows, replace=False))
+        kind = O.MASK_TEMPORAL if kinds[h] == 1 else O.MASK_SPATIAL
+        t0 = time.perf_counter()
+        pi = O.permutation(wl.T, wl.P, wl.n_text)
+        lrows = pi[rows] if kind == O.MASK_TEMPORAL else rows
+        qblocks = sorted(set((lrows // wl.block_q).tolist()))
+        bm_rows = O.block_mask_rows(kind, qblocks, wl.T, wl.P, wl.n_text, wl.spatial_band,
+                                    wl.temporal_width, wl.block_q, wl.block_k)
+        bm = np.zeros(( -(-wl.N // wl.block_q), bm_rows.shape[1]), dtype=bool)
+        bm[qblocks] = bm_rows
+        O.layer_rows(q, k, v, kinds[h], wl.T, wl.P, wl.n_text, wl.spatial_band,
+                     wl.temporal_width, wl.block_q, wl.block_k, wl.scale, rows=rows, bm=bm)
+        elapsed += time.perf_counter() - t0
+        cols_in = np.minimum(wl.block_k, wl.N - np.arange(bm.shape[1]) * wl.block_k)
+        for r in lrows:
+            flops += 4 * wl.d * int(np.sum(cols_in[bm[r // wl.block_q]]))
+    return elapsed, flops
+
+
+def cpu_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, wl):
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return
+    heads = [h for h, kd in enumerate(SI.planted_head_kinds(wl)) if kd == 0][:1] + \
+            [h for h, kd in enumerate(SI.planted_head_kinds(wl)) if kd == 1][:1]
+    n_rows = 24
+    for _ in range(args.warmup):
+        oracle_sample(wl, 4, heads[:1])
+    times, flops = [], 0
+    for s in range(args.steps):
+        t, f = oracle_sample(wl, n_rows, heads, seed=100 + s)
+        times.append(t)
+        flops = f
+    ms = 1e3 * statistics.mean(times)
+    value = flops / (ms * 1e-3) / 1e12
+    sample = (f"fp64 oracle attention output of {n_rows} query rows x {len(heads)} heads "
+              f"(one spatial, one temporal) of {wl.name} per step, with their block-mask rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(SI.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    wl = SI.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    import video_dit_spatial_b200 as svg
+    from video_dit_spatial_b200.layer import SparseVideoGenLayer
+    svg.load()
+    g = svg.Geom.from_workload(wl)
+    dev = torch.device("cuda", local)
+
+    # inputs: generated on the host (seeded per rank), pinned, copied once
+    wl_r = wl.replace(seed=wl.seed + 7919 * rank) if rank else wl
+    qh, kh, vh = (t.pin_memory() for t in SI.make_qkv(wl_r))
+    rows_h = SI.sample_rows(wl).pin_memory()
+    q, k, v = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
+    rows = rows_h.to(dev)
+    o = torch.empty_like(q)
+    layer = SparseVideoGenLayer(g, wl.n_samples, dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(q, k, v, rows, o, rebuild_masks=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # algorithmic work of one step (computed-block pairs by each head's label)
+    labels = layer.labels.cpu().numpy()
+    pairs = {kind: computed_pairs(svg, g, kind) for kind in (0, 1)}
+    attn_flops = sum(4 * wl.d * pairs[int(lb)] for lb in labels)
+    dense_flops = 4 * wl.d * wl.N * wl.N * wl.B * wl.H
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clock_info = clocks.stop() if clocks else None
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    gpu_launches = 7 * args.steps  # profile, finalize, 2 masks, permute_qkv, attention, unpermute
+
+    # per-kernel timing (events on the launch stream), then the dense baseline
+    def time_fn(fn, reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms_profile = time_fn(lambda: layer.profile(q, k, v, rows), 5)
+    ms_masks = time_fn(layer.build_masks, 5)
+    ms_permute = time_fn(lambda: svg.svg_permute_qkv(g, q, k, v, layer.qp, layer.kp, layer.vp,
+                                                     layer.labels), 5)
+    ms_unpermute = time_fn(lambda: svg.svg_unpermute(g, layer.op, o, layer.labels), 5)
+    ms_attn = time_fn(lambda: svg.svg_sparse_attention(
+        g, q, k, v, layer.qp, layer.kp, layer.vp, layer.labels,
+        layer.masks[0].row_ptr, layer.masks[0].col_idx, layer.masks[1].row_ptr,
+        layer.masks[1].col_idx, o, layer.op), max(3, args.steps))
+    ms_dense = None
+    if not args.no_dense:
+        od = torch.empty_like(q)
+        ms_dense = time_fn(lambda: layer.dense(q, k, v, od), 2)
+        del od
+    st, bits = svg.svg_get_device_status()
+    if st != svg.SVG_OK:
+        raise RuntimeError(f"device status {st} bits {bits}")
+
+    # end to end through the public API: pinned host inputs -> device -> host result
+    e2e = None
+    if not args.no_e2e:
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, rows_h))
+        d2h = o_h.numel() * o_h.element_size()
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            rows.copy_(rows_h, non_blocking=True)
+            layer.forward(q, k, v, rows, o, rebuild_masks=True)
+            o_h.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(2, min(args.steps, 5))
+        e0.record(stream)
+        for _ in range(reps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / reps
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * attn_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    pk = _peaks()
+    achieved = attn_flops / (ms_attn * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "sparse_attention_kernel", "achieved": achieved,
+                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops_sustained"],
+                "peak_kind": f"bf16 dense, sustained, {pk['source']}",
+                "frac_of_burst_peak": achieved / pk["bf16_tflops"],
+                "traffic": None}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        kinds = SI.planted_head_kinds(wl)
+        heads = [kinds.index(0), kinds.index(1)]
+        secs, fl = oracle_sample(wl, 24, heads)
+        cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"fp64 oracle attention output of 24 query rows x 2 heads (one spatial, "
+                         f"one temporal) of {wl.name}, with their block-mask rows",
+               "seconds": secs}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * attn_flops / (ms * 1e-3) / 1e12, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d,
+                       "T": wl.T, "P": wl.P, "n_text": wl.n_text, "block": wl.block_q,
+                       "spatial_band": wl.spatial_band, "temporal_width": wl.temporal_width,
+                       "n_samples": wl.n_samples,
+                       "l2": "inputs larger than L2 (Q,K,V %.2f GB)" % (3 * q.numel() * 2 / 1e9),
+                       "parallelism": f"independent replicas x{world}" if world > 1 else "1 GPU"},
+            "layer_ms": ms,
+            "attn_ms": ms_attn, "dense_ms": ms_dense,
+            "speedup_vs_dense": (ms_dense / ms_attn) if ms_dense else None,
+            "layer_speedup_vs_dense": (ms_dense / ms) if ms_dense else None,
+            "attn_tflops": achieved,
+            "dense_tflops": (dense_flops / (ms_dense * 1e-3) / 1e12) if ms_dense else None,
+            "kernel_ms": {"profile": ms_profile, "block_masks": ms_masks,
+                          "permute_qkv": ms_permute, "attention": ms_attn,
+                          "unpermute": ms_unpermute},
+            "labels_temporal": int(np.sum(labels == 1)),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": gpu_launches, "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+/*
+ * svg.h -- C ABI of libsvg, a B200 (sm_100a) implementation of the hot path of
+ * Sparse VideoGen (SVG 1) spatial/temporal sparse 3D attention.
+ *
+ * Source of the method: "Sparse VideoGen: Accelerating Video Diffusion
+ * Transformers with Spatial-Temporal Sparsity" (arXiv 2502.01776), abstract:
+ * attention heads of a video diffusion transformer are classified online as
+ * spatial heads (output dominated by tokens of the query's own and nearby
+ * frames) or temporal heads (dominated by tokens at the same in-frame position
+ * across frames); a hardware-efficient tensor layout transformation and
+ * customised kernels turn either pattern into contiguous block-sparse work.
+ * The project article "Sparse-VideoGen and the sparsity hiding inside video
+ * diffusion attention" (section "Three generations of the same idea", and the
+ * install section on block sparse attention with varied block sizes) restates
+ * the same pieces. The pages fix no interface; this one is derived from that
+ * description.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  Tensors   Q, K, V, O are [B, H, N, d] bf16 (raw bit patterns, svg_bf16),
+ *            contiguous, base address 16-byte aligned, N = T*P + n_text.
+ *            Video token (frame f, position p) is row f*P + p in frame-major
+ *            order and row p*T + f in position-major order; the n_text text
+ *            tokens follow the video tokens in both orders and are global.
+ *  Memory    All pointers marked "device" are caller-owned device memory; the
+ *            library allocates no device memory and frees nothing. Each
+ *            attention/profiling CTA allocates and frees its own tensor memory.
+ *  Streams   Every call that takes a stream enqueues its work on that stream
+ *            (a cudaStream_t passed as void*; NULL = legacy default stream)
+ *            and returns without synchronising.
+ *  Errors    Every call returns an svg_status. Arguments are validated on the
+ *            host before anything is launched; on any error nothing is
+ *            launched and outputs are untouched. Nothing aborts, traps or
+ *            prints. Device-side waits are bounded: one that runs out sets a
+ *            status bit read by svg_get_device_status.
+ *  Devices   The current CUDA device at call time must be an sm_100 GPU
+ *            (SVG_ERR_UNSUPPORTED otherwise).
+ */
+#ifndef SVG_H_
+#define SVG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svg_status {
+  SVG_OK = 0,
+  SVG_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned tensor, bad kind */
+  SVG_ERR_UNSUPPORTED = 2,   /* head_dim not in {64,128}, block size not in {64,128},
+                                not an sm_100 device */
+  SVG_ERR_CAPACITY = 3,      /* caller buffer too small (col_capacity, workspace) */
+  SVG_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  SVG_ERR_DEVICE_TIMEOUT = 5 /* a device-side bounded wait ran out (see svg_get_device_status) */
+} svg_status;
+
+/* Head labels (one int8 per (b, h), index b*H + h). */
+enum { SVG_HEAD_SPATIAL = 0, SVG_HEAD_TEMPORAL = 1 };
+
+/* Block-mask kinds. SPATIAL lives in frame-major order, TEMPORAL in
+ * position-major order, DENSE (all blocks) in either. */
+enum { SVG_MASK_SPATIAL = 0, SVG_MASK_TEMPORAL = 1, SVG_MASK_DENSE = 2 };
+
+typedef uint16_t svg_bf16; /* raw bf16 bits */
+typedef void* svg_stream_t; /* a cudaStream_t */
+
+/* Geometry of one attention layer. */
+typedef struct svg_geom {
+  int32_t B, H;            /* batch, heads (>= 1) */
+  int32_t T, P;            /* frames, tokens per frame (>= 1) */
+  int32_t n_text;          /* text tokens after the T*P video tokens (>= 0) */
+  int32_t head_dim;        /* d: 64 or 128 */
+  int32_t block_q;         /* query block rows of the block mask: 64 or 128 */
+  int32_t block_k;         /* key block columns of the block mask: 64 or 128 */
+  int32_t spatial_band;    /* s >= 0: spatial mask keeps key frames with |f(i)-f(j)| <= s */
+  int32_t temporal_width;  /* w >= 0: temporal mask keeps in-frame positions |p(i)-p(j)| <= w */
+  float scale;             /* softmax scale applied to q.k (normally 1/sqrt(d)); finite, > 0 */
+} svg_geom;
+
+/* ---------------------------------------------------------------------------
+ * svg_mask_nnz -- host only, exact.
+ * Number of (query block, key block) pairs of the block mask `kind` (the
+ * length col_idx must have for svg_build_block_mask). Block (r, c) is on iff
+ * some token pair of the block pair is allowed by the token mask in the
+ * pattern's layout (SVG abstract: spatial heads attend within nearby frames,
+ * temporal heads across frames at nearby positions; text tokens are global).
+ *   nnz  out, host pointer.
+ * Errors: INVALID_ARG (null, bad geometry, bad kind).
+ */
+svg_status svg_mask_nnz(const svg_geom* geom, int32_t kind, int64_t* nnz);
+
+/* ---------------------------------------------------------------------------
+ * svg_build_block_mask -- the block mask of `kind` as CSR.
+ *   row_ptr   device int32 [nQB + 1], nQB = ceil(N / block_q); row_ptr[0] = 0.
+ *   col_idx   device int32 [col_capacity]; key-block indices of each row,
+ *             ascending; nnz = row_ptr[nQB] = svg_mask_nnz(...).
+ * Built in closed form: a query block's video tokens span an integer interval
+ * of frames (spatial) or positions (temporal), so each row is one contiguous
+ * run of key blocks plus the text key blocks. Depends only on the geometry;
+ * callers build it once and reuse it across layers and steps.
+ * Errors: INVALID_ARG, CAPACITY (col_capacity < nnz), CUDA.
+ */
+svg_status svg_build_block_mask(const svg_geom* geom, int32_t kind, int32_t* row_ptr,
+                                int32_t* col_idx, int64_t col_capacity, svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * svg_profile_workspace_bytes -- host only: device workspace svg_profile_heads
+ * needs for n_samples sampled rows (partial sums of the MSE reduction).
+ */
+svg_status svg_profile_workspace_bytes(const svg_geom* geom, int32_t n_samples, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * svg_profile_heads -- online profiling (SVG abstract: "online profiling
+ * strategy to capture the dynamic sparse patterns and predict the type of
+ * attention head").
+ * For every (b, h) and every sampled query row i, computes full attention,
+ * spatial-masked attention (|f(i)-f(j)| <= s, text global) and
+ * temporal-masked attention (|p(i)-p(j)| <= w, text global), all token-level
+ * in frame-major order, then
+ *   mse_X = mean over rows x channels of (O_X - O_full)^2,
+ *   label = SVG_HEAD_TEMPORAL iff mse_temporal < mse_spatial (tie: spatial).
+ *   q, k, v      device bf16 [B, H, N, d], frame-major.
+ *   sample_idx   device int32 [n_samples], distinct video rows in [0, T*P);
+ *                the same rows serve every (b, h).
+ *   labels       device int8 [B*H], out.
+ *   mse          device float [B*H*2] out ({spatial, temporal} per head), or NULL.
+ *   workspace    device, >= svg_profile_workspace_bytes(...), 256-byte aligned.
+ * Deterministic: fixed-order reductions, no atomics in the arithmetic.
+ * Errors: INVALID_ARG, UNSUPPORTED, CAPACITY (workspace too small), CUDA.
+ * A sample index outside [0, T*P) sets the device bounds bit (row skipped).
+ */
+svg_status svg_profile_heads(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                             const svg_bf16* v, const int32_t* sample_idx, int32_t n_samples,
+                             int8_t* labels, float* mse, void* workspace,
+                             size_t workspace_bytes, svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * svg_permute / svg_unpermute -- the layout transformation (SVG abstract:
+ * "hardware-efficient tensor layout transformation").
+ *   permute:    out[b,h,pi(i),:] = in[b,h,i,:]   (frame-major -> position-major)
+ *   unpermute:  out[b,h,i,:]     = in[b,h,pi(i),:]
+ * with pi(f*P + p) = p*T + f for video rows and pi(i) = i for text rows.
+ *   in, out   device bf16 [B, H, N, d]; must not overlap.
+ *   labels    device int8 [B*H]: only heads labelled SVG_HEAD_TEMPORAL are
+ *             written (others untouched); NULL = every head.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+svg_status svg_permute(const svg_geom* geom, const svg_bf16* in, svg_bf16* out,
+                       const int8_t* labels, svg_stream_t stream);
+svg_status svg_unpermute(const svg_geom* geom, const svg_bf16* in, svg_bf16* out,
+                         const int8_t* labels, svg_stream_t stream);
+
+/* svg_permute_qkv -- svg_permute of Q, K and V in one launch. */
+svg_status svg_permute_qkv(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                           const svg_bf16* v, svg_bf16* qp, svg_bf16* kp, svg_bf16* vp,
+                           const int8_t* labels, svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * svg_sparse_attention -- block-sparse flash attention over per-head block
+ * masks (SVG abstract: "customized kernel implementations"; the project
+ * article's block sparse attention).
+ * Head (b, h) with label l works in layout L(l): frame-major for spatial
+ * heads (reads q, k, v; CSR row_ptr_s/col_idx_s; writes o), position-major
+ * for temporal heads (reads qp, kp, vp; CSR row_ptr_t/col_idx_t; writes op).
+ * For each query row i of the head:
+ *   O[i] = sum_{j < N, BM[i/block_q][j/block_k] = 1} softmax_j(scale * q_i.k_j) v_j
+ * (block-granular: every token pair of a listed block pair is attended),
+ * accumulated in fp32, rounded to bf16. Rows whose CSR row is empty get O = 0.
+ *   q,k,v,o        device bf16 [B,H,N,d] (frame-major).
+ *   qp,kp,vp,op    device bf16 [B,H,N,d] (position-major); may be NULL when
+ *                  labels is NULL or no head is temporal (then a temporal
+ *                  label sets the device bounds bit and the head is skipped).
+ *   labels         device int8 [B*H]; NULL = every head spatial.
+ *   row_ptr_*, col_idx_*  device CSR as built by svg_build_block_mask (any CSR
+ *                  with ascending, in-range column indices is accepted;
+ *                  out-of-range indices set the bounds bit and are skipped).
+ *                  The temporal CSR may be NULL when labels is NULL.
+ *   lse            device float [B,H,N] out (natural-log sum of exp of the
+ *                  scaled logits over attended keys, in the head's layout;
+ *                  -inf for empty rows), or NULL.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+svg_status svg_sparse_attention(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                                const svg_bf16* v, const svg_bf16* qp, const svg_bf16* kp,
+                                const svg_bf16* vp, const int8_t* labels,
+                                const int32_t* row_ptr_s, const int32_t* col_idx_s,
+                                const int32_t* row_ptr_t, const int32_t* col_idx_t,
+                                svg_bf16* o, svg_bf16* op, float* lse, svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * svg_get_device_status -- synchronises `stream`, then reads and clears the
+ * device status bits of the current device (1 = a bounded wait ran out,
+ * 2 = an out-of-range index from caller memory was skipped) into *bits
+ * (may be NULL). Returns SVG_ERR_DEVICE_TIMEOUT if bit 1 was set,
+ * SVG_ERR_INVALID_ARG if only bit 2 was set, SVG_ERR_CUDA on a CUDA error
+ * (including errors of earlier asynchronous launches), SVG_OK otherwise.
+ */
+svg_status svg_get_device_status(svg_stream_t stream, int32_t* bits);
+
+/* ---------------------------------------------------------------------------
+ * svg_selftest_wait_timeout -- failure-detection self-test. Launches one CTA
+ * whose thread waits, through the same bounded wait the kernels use, on a
+ * shared-memory barrier that nothing ever completes, with a limit of
+ * limit_cycles SM clock cycles (1 .. 2^31). The wait runs out, sets the
+ * timeout status bit and the kernel returns normally; no fault, trap or hang.
+ */
+svg_status svg_selftest_wait_timeout(int64_t limit_cycles, svg_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* svg_status_string(svg_status status);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int32_t svg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVG_H_ */

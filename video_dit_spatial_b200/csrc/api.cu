@@ -1,0 +1,367 @@
+// C ABI of libsvg (declared in include/svg.h): argument validation, geometry,
+// tensor-map encoding and the launches of the kernels in the other
+// translation units. Every entry point validates everything on the host
+// before it launches anything.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace svg {
+
+// Status word of this module: device kernels OR error bits into it; the host
+// passes its address to every kernel and reads it back in
+// svg_get_device_status.
+__device__ int g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+int* g_status_ptr[kMaxDevices] = {};
+int g_is_sm100[kMaxDevices] = {};  // 0 unknown, 1 yes, -1 no
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+inline bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+svg_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVG_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SVG_ERR_UNSUPPORTED;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_is_sm100[dev] != 0) return g_is_sm100[dev] > 0 ? SVG_OK : SVG_ERR_UNSUPPORTED;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SVG_ERR_CUDA;
+  const bool ok = major == 10 && minor == 0;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_is_sm100[dev] = ok ? 1 : -1;
+  return ok ? SVG_OK : SVG_ERR_UNSUPPORTED;
+}
+
+// Geometry checks shared by every entry point. `need_kernel_shape` also asks
+// for the head dims / block sizes the kernels are built for.
+svg_status check_geom(const svg_geom* g, bool need_kernel_shape) {
+  if (g == nullptr) return SVG_ERR_INVALID_ARG;
+  if (g->B < 1 || g->H < 1 || g->T < 1 || g->P < 1 || g->n_text < 0) return SVG_ERR_INVALID_ARG;
+  if (g->spatial_band < 0 || g->temporal_width < 0) return SVG_ERR_INVALID_ARG;
+  if (g->block_q < 1 || g->block_k < 1 || g->head_dim < 1) return SVG_ERR_INVALID_ARG;
+  const int64_t N = static_cast<int64_t>(g->T) * g->P + g->n_text;
+  if (N > (static_cast<int64_t>(1) << 30)) return SVG_ERR_INVALID_ARG;
+  const int64_t BH = static_cast<int64_t>(g->B) * g->H;
+  if (BH > 65535) return SVG_ERR_INVALID_ARG;
+  if (!(g->scale > 0.0f) || !(g->scale < 3.0e38f)) return SVG_ERR_INVALID_ARG;
+  if (need_kernel_shape) {
+    if (g->head_dim != 64 && g->head_dim != 128) return SVG_ERR_UNSUPPORTED;
+    if ((g->block_q != 64 && g->block_q != 128) || (g->block_k != 64 && g->block_k != 128))
+      return SVG_ERR_UNSUPPORTED;
+    const int64_t nqb = (N + g->block_q - 1) / g->block_q;
+    if (nqb > 0x7fffffff) return SVG_ERR_INVALID_ARG;
+  }
+  return SVG_OK;
+}
+
+int64_t mask_nnz_host(const Dims& d, int32_t kind) {
+  const MaskGeom m = make_mask_geom(d, kind);
+  int64_t nnz = 0;
+  for (int32_t r = 0; r < d.nqb; ++r) nnz += mask_row(m, r).count();
+  return nnz;
+}
+
+}  // namespace
+
+Dims make_dims(const svg_geom& g) {
+  Dims d;
+  d.B = g.B;
+  d.H = g.H;
+  d.BH = g.B * g.H;
+  d.T = g.T;
+  d.P = g.P;
+  d.n_text = g.n_text;
+  d.d = g.head_dim;
+  d.bq = g.block_q;
+  d.bk = g.block_k;
+  d.s = g.spatial_band;
+  d.w = g.temporal_width;
+  d.Nv = g.T * g.P;
+  d.N = d.Nv + g.n_text;
+  d.nqb = (d.N + d.bq - 1) / d.bq;
+  d.nkb = (d.N + d.bk - 1) / d.bk;
+  d.scale = g.scale;
+  return d;
+}
+
+int* device_status_word(cudaError_t* err) {
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_status_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    *err = cudaGetSymbolAddress(&ptr, g_device_status);
+    if (*err != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(ptr);
+  }
+  return g_status_ptr[dev];
+}
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int32_t d, int32_t N, int32_t BH,
+                    int32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace svg
+
+using svg::Dims;
+
+extern "C" {
+
+const char* svg_status_string(svg_status s) {
+  switch (s) {
+    case SVG_OK: return "SVG_OK";
+    case SVG_ERR_INVALID_ARG: return "SVG_ERR_INVALID_ARG";
+    case SVG_ERR_UNSUPPORTED: return "SVG_ERR_UNSUPPORTED";
+    case SVG_ERR_CAPACITY: return "SVG_ERR_CAPACITY";
+    case SVG_ERR_CUDA: return "SVG_ERR_CUDA";
+    case SVG_ERR_DEVICE_TIMEOUT: return "SVG_ERR_DEVICE_TIMEOUT";
+  }
+  return "SVG_ERR_UNKNOWN";
+}
+
+int32_t svg_version(void) { return 100; }
+
+svg_status svg_mask_nnz(const svg_geom* geom, int32_t kind, int64_t* nnz) {
+  if (nnz == nullptr) return SVG_ERR_INVALID_ARG;
+  if (kind < SVG_MASK_SPATIAL || kind > SVG_MASK_DENSE) return SVG_ERR_INVALID_ARG;
+  const svg_status st = svg::check_geom(geom, false);
+  if (st != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  *nnz = svg::mask_nnz_host(d, kind);
+  return SVG_OK;
+}
+
+svg_status svg_build_block_mask(const svg_geom* geom, int32_t kind, int32_t* row_ptr,
+                                int32_t* col_idx, int64_t col_capacity, svg_stream_t stream) {
+  if (row_ptr == nullptr || col_idx == nullptr) return SVG_ERR_INVALID_ARG;
+  if (kind < SVG_MASK_SPATIAL || kind > SVG_MASK_DENSE) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_geom(geom, false);
+  if (st != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  const int64_t nnz = svg::mask_nnz_host(d, kind);
+  if (nnz > 0x7fffffffLL) return SVG_ERR_INVALID_ARG;
+  if (col_capacity < nnz) return SVG_ERR_CAPACITY;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  if (svg::launch_block_mask(d, kind, row_ptr, col_idx, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SVG_ERR_CUDA;
+  return SVG_OK;
+}
+
+svg_status svg_profile_workspace_bytes(const svg_geom* geom, int32_t n_samples, size_t* bytes) {
+  if (bytes == nullptr || n_samples < 1) return SVG_ERR_INVALID_ARG;
+  const svg_status st = svg::check_geom(geom, false);
+  if (st != SVG_OK) return st;
+  const size_t BH = static_cast<size_t>(geom->B) * geom->H;
+  *bytes = BH * 2 * static_cast<size_t>(svg::profile_tiles(n_samples)) * sizeof(float);
+  return SVG_OK;
+}
+
+svg_status svg_profile_heads(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                             const svg_bf16* v, const int32_t* sample_idx, int32_t n_samples,
+                             int8_t* labels, float* mse, void* workspace, size_t workspace_bytes,
+                             svg_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || sample_idx == nullptr ||
+      labels == nullptr || workspace == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  if (!svg::aligned16(q) || !svg::aligned16(k) || !svg::aligned16(v)) return SVG_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_geom(geom, true);
+  if (st != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  if (n_samples < 1 || n_samples > d.Nv) return SVG_ERR_INVALID_ARG;
+  size_t need = 0;
+  svg_profile_workspace_bytes(geom, n_samples, &need);
+  if (workspace_bytes < need) return SVG_ERR_CAPACITY;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  svg::ProfileArgs a{q, k, v, sample_idx, n_samples, labels, mse, static_cast<float*>(workspace)};
+  if (svg::launch_profile(d, a, status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SVG_ERR_CUDA;
+  return SVG_OK;
+}
+
+static svg_status permute_common(const svg_geom* geom, int n, const svg_bf16* const* in,
+                                 svg_bf16* const* out, const int8_t* labels, bool inverse,
+                                 svg_stream_t stream) {
+  svg_status st = svg::check_geom(geom, false);
+  if (st != SVG_OK) return st;
+  if (geom->head_dim != 64 && geom->head_dim != 128) return SVG_ERR_UNSUPPORTED;
+  const Dims d = svg::make_dims(*geom);
+  const size_t bytes = static_cast<size_t>(d.BH) * d.N * d.d * 2;
+  for (int t = 0; t < n; ++t) {
+    if (in[t] == nullptr || out[t] == nullptr) return SVG_ERR_INVALID_ARG;
+    if (!svg::aligned16(in[t]) || !svg::aligned16(out[t])) return SVG_ERR_INVALID_ARG;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(in[t]), b0 = reinterpret_cast<uintptr_t>(out[t]);
+    if (a0 < b0 + bytes && b0 < a0 + bytes) return SVG_ERR_INVALID_ARG;  // overlap
+  }
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  if (svg::launch_permute(d, n, in, out, labels, inverse, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SVG_ERR_CUDA;
+  return SVG_OK;
+}
+
+svg_status svg_permute(const svg_geom* geom, const svg_bf16* in, svg_bf16* out,
+                       const int8_t* labels, svg_stream_t stream) {
+  const svg_bf16* i[1] = {in};
+  svg_bf16* o[1] = {out};
+  return permute_common(geom, 1, i, o, labels, false, stream);
+}
+
+svg_status svg_unpermute(const svg_geom* geom, const svg_bf16* in, svg_bf16* out,
+                         const int8_t* labels, svg_stream_t stream) {
+  const svg_bf16* i[1] = {in};
+  svg_bf16* o[1] = {out};
+  return permute_common(geom, 1, i, o, labels, true, stream);
+}
+
+svg_status svg_permute_qkv(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                           const svg_bf16* v, svg_bf16* qp, svg_bf16* kp, svg_bf16* vp,
+                           const int8_t* labels, svg_stream_t stream) {
+  const svg_bf16* i[3] = {q, k, v};
+  svg_bf16* o[3] = {qp, kp, vp};
+  return permute_common(geom, 3, i, o, labels, false, stream);
+}
+
+svg_status svg_sparse_attention(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                                const svg_bf16* v, const svg_bf16* qp, const svg_bf16* kp,
+                                const svg_bf16* vp, const int8_t* labels,
+                                const int32_t* row_ptr_s, const int32_t* col_idx_s,
+                                const int32_t* row_ptr_t, const int32_t* col_idx_t, svg_bf16* o,
+                                svg_bf16* op, float* lse, svg_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || row_ptr_s == nullptr ||
+      col_idx_s == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  const bool any_perm = qp || kp || vp || op;
+  const bool all_perm = qp && kp && vp && op;
+  if (any_perm && !all_perm) return SVG_ERR_INVALID_ARG;
+  if (all_perm && (row_ptr_t == nullptr || col_idx_t == nullptr)) return SVG_ERR_INVALID_ARG;
+  const svg_bf16* tensors[8] = {q, k, v, o, qp, kp, vp, op};
+  for (int t = 0; t < 8; ++t)
+    if (tensors[t] != nullptr && !svg::aligned16(tensors[t])) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_geom(geom, true);
+  if (st != SVG_OK) return st;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  svg::AttnArgs a{q, k, v, qp, kp, vp, labels, row_ptr_s, col_idx_s, row_ptr_t, col_idx_t,
+                  o, op, lse};
+  if (svg::launch_sparse_attention(d, a, status, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SVG_ERR_CUDA;
+  return SVG_OK;
+}
+
+svg_status svg_get_device_status(svg_stream_t stream, int32_t* bits) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SVG_ERR_CUDA;
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  int value = 0;
+  if (cudaMemcpyFromSymbol(&value, svg::g_device_status, sizeof(int)) != cudaSuccess)
+    return SVG_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(svg::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+    return SVG_ERR_CUDA;
+  if (bits != nullptr) *bits = value;
+  if (value & svg::kDevErrTimeout) return SVG_ERR_DEVICE_TIMEOUT;
+  if (value & svg::kDevErrBounds) return SVG_ERR_INVALID_ARG;
+  return SVG_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- self-test
+namespace svg {
+namespace {
+__global__ void wait_selftest_kernel(long long limit, int* status) {
+  __shared__ uint64_t never;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&never, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Same loop shape as mbar_wait, with a caller-chosen limit.
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&never, 0)) {
+      if (clock64() - t0 > limit) {
+        abort_flag = 1;
+        atomicOr(status, kDevErrTimeout);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(long long limit_cycles, int* status, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_cycles, status);
+  return cudaGetLastError();
+}
+}  // namespace svg
+
+extern "C" svg_status svg_selftest_wait_timeout(int64_t limit_cycles, svg_stream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > (static_cast<int64_t>(1) << 31)) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  if (svg::launch_wait_selftest(limit_cycles, status, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SVG_ERR_CUDA;
+  return SVG_OK;
+}

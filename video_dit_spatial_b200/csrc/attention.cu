@@ -1,0 +1,419 @@
+// Block-sparse flash attention of Sparse VideoGen (arXiv 2502.01776 abstract:
+// "customized kernel implementations" for the spatial/temporal sparse 3D
+// attention; the project article "Sparse-VideoGen and the sparsity hiding
+// inside video diffusion attention" names block sparse attention with varied
+// block sizes). For every query block the kernel walks that block's CSR list of
+// key blocks; every listed (query block, key block) pair is attended in full.
+//
+// One CTA = one (b*H + h, query block). 192 threads, warp-specialised:
+//   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
+//   warp 4     TMA producer: the Q tile once, then K/V tiles of the listed
+//              key blocks into a ring of shared-memory stages
+//   warp 5     MMA issuer (one thread): S = Q K^T (both operands in shared
+//              memory, 128-byte swizzle) and O += P V (P from tensor memory,
+//              V from shared memory) with tcgen05.mma, fp32 accumulators in
+//              tensor memory
+// Tensor memory (512 columns): S double buffer at columns 0 and 128, O at 256.
+// P (bf16) overwrites the first half of its S buffer. While the softmax warps
+// work on S_j the tensor core already computes S_{j+1}; P_j V_j follows as
+// soon as P_j is written. The running maximum is re-based lazily (only when
+// a tile's maximum exceeds it by more than 2^8), so O is rarely rescaled.
+// All barrier waits are bounded (see sm100.cuh).
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace svg {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr float kRebaseLog2 = 8.0f;  // lazy re-basing threshold (log2 units)
+
+template <int D, int BK>
+struct Cfg {
+  static constexpr int kPanels = D / 64;            // 128-byte wide column panels
+  static constexpr int kQPanel = 128 * 128;         // 128 rows x 128 B
+  static constexpr int kKVPanel = BK * 128;         // BK rows x 128 B
+  static constexpr int kQBytes = kPanels * kQPanel;
+  static constexpr int kKVBytes = kPanels * kKVPanel;  // one K (or V) tile
+  static constexpr int kStages = D == 128 ? 2 : 3;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kUsed = kOffBar + kBarBytes + 1024;  // + alignment slack
+  // Keep one CTA per SM: each CTA takes all 512 tensor-memory columns.
+  static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+};
+
+struct __align__(64) AttnParams {
+  CUtensorMap tm_q[2], tm_k[2], tm_v[2];  // [0]: frame-major, [1]: position-major
+  const int8_t* labels;
+  const int32_t* row_ptr[2];
+  const int32_t* col_idx[2];
+  svg_bf16* out[2];
+  float* lse;
+  int* status;
+  int32_t N, BH, nqb, nkb, bq, bk;
+  int32_t has_permuted;
+  float scale_log2;
+};
+
+struct Barriers {
+  uint64_t q_full;
+  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full, o_final, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attention_kernel(const __grid_constant__ AttnParams p) {
+  using C = Cfg<D, BK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  Barriers* bar = reinterpret_cast<Barriers*>(smem + C::kOffBar);
+  volatile int* abort_flag = &bar->abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int qb = p.nqb - 1 - static_cast<int>(blockIdx.x);  // text-heavy (longest) rows first
+  const int bh = blockIdx.y;
+
+  const int label = p.labels ? static_cast<int>(p.labels[bh]) : SVG_HEAD_SPATIAL;
+  const int sel = label == SVG_HEAD_TEMPORAL ? 1 : 0;
+  if (label != SVG_HEAD_SPATIAL && label != SVG_HEAD_TEMPORAL) {
+    if (tid == 0) atomicOr(p.status, kDevErrBounds);
+    return;
+  }
+  if (sel == 1 && !p.has_permuted) {
+    if (tid == 0) atomicOr(p.status, kDevErrBounds);
+    return;
+  }
+  const int32_t rp0 = __ldg(p.row_ptr[sel] + qb);
+  int32_t n = __ldg(p.row_ptr[sel] + qb + 1) - rp0;
+  if (n < 0 || n > p.nkb) {
+    if (tid == 0) atomicOr(p.status, kDevErrBounds);
+    n = 0;
+  }
+  const int32_t* cols = p.col_idx[sel] + rp0;
+
+  // ---- set-up: barriers, tensor memory, padding rows of a short Q tile
+  if (warp == 0) {
+    tmem_alloc(&bar->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 32) {
+    mbar_init(&bar->q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->s_full[s], 1);
+      mbar_init(&bar->p_full[s], 128);
+    }
+    mbar_init(&bar->o_full, 1);
+    mbar_init(&bar->o_final, 1);
+    mbar_init(&bar->drain, 1);
+    bar->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (p.bq < 128 && tid < 128 && tid >= p.bq) {
+    for (int pn = 0; pn < C::kPanels; ++pn) {
+      uint4* row = reinterpret_cast<uint4*>(sQ + pn * C::kQPanel + tid * 128);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) row[i] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane_id() == 0 && n > 0) {
+      const CUtensorMap* mq = &p.tm_q[sel];
+      const CUtensorMap* mk = &p.tm_k[sel];
+      const CUtensorMap* mv = &p.tm_v[sel];
+      const uint64_t keep = l2_policy_evict_last();
+      mbar_arrive_expect_tx(&bar->q_full, static_cast<uint32_t>(p.bq * D * 2));
+      for (int pn = 0; pn < C::kPanels; ++pn)
+        tma_load_3d(sQ + pn * C::kQPanel, mq, &bar->q_full, pn * 64, qb * p.bq, bh);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % C::kStages;
+        if (!mbar_wait(&bar->kv_empty[st], ((j / C::kStages) & 1) ^ 1, abort_flag, p.status))
+          break;
+        int c = __ldg(cols + j);
+        if (c < 0 || c >= p.nkb) c = 0;  // flagged and masked by the softmax warps
+        mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kKVPanel, mk, &bar->k_full[st],
+                           pn * 64, c * BK, bh, keep);
+        mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kKVPanel, mv, &bar->v_full[st],
+                           pn * 64, c * BK, bh, keep);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        // Let every copy this thread started land before the CTA retires.
+        for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
+          const int st = j % C::kStages;
+          const uint32_t par = (j / C::kStages) & 1;
+          int spare = 0;
+          long long t0 = clock64();
+          while (!(mbar_try_wait(&bar->k_full[st], par) && mbar_try_wait(&bar->v_full[st], par)) &&
+                 clock64() - t0 < kWaitLimitCycles)
+            ++spare;
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane_id() == 0 && n > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BK, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t k_addr = smem_u32(sK);
+      const uint32_t v_addr = smem_u32(sV);
+      bool ok = mbar_wait(&bar->q_full, 0, abort_flag, p.status);
+      tc_fence_after();
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % C::kStages;
+          const uint32_t s_col = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
+          if (!mbar_wait(&bar->k_full[st], (j / C::kStages) & 1, abort_flag, p.status)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;  // 16 bf16 of K inside the 128-byte row
+            const uint64_t a = sdesc_sw128(q_addr + (kk >> 2) * C::kQPanel + off, 16, 1024);
+            const uint64_t b =
+                sdesc_sw128(k_addr + st * C::kKVBytes + (kk >> 2) * C::kKVPanel + off, 16, 1024);
+            mma_bf16_ss(s_col, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bar->s_full[j & 1]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int st = jj % C::kStages;
+          const uint32_t p_col = tmem + ((jj & 1) ? C::kColS1 : C::kColS0);
+          if (!mbar_wait(&bar->p_full[jj & 1], (jj >> 1) & 1, abort_flag, p.status)) break;
+          if (!mbar_wait(&bar->v_full[st], (jj / C::kStages) & 1, abort_flag, p.status)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t b = sdesc_sw128(v_addr + st * C::kKVBytes + kk * 16 * 128,
+                                           C::kKVPanel, 1024);
+            mma_bf16_ts(tmem + C::kColO, p_col + kk * 8, b, idesc_pv,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&bar->kv_empty[st]);
+          tc_commit(&bar->o_full);
+          if (jj == n - 1) tc_commit(&bar->o_final);
+        }
+      }
+      if (*abort_flag) {
+        // Retire every MMA issued so far before tensor memory is released.
+        tc_commit(&bar->drain);
+        long long t0 = clock64();
+        while (!mbar_try_wait(&bar->drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int row = qb * p.bq + tid;
+    const bool row_valid = tid < p.bq && row < p.N;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m = -INFINITY;  // running base, log2 units
+    float l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int sb = j & 1;
+      const uint32_t s_col = lane_base + (sb ? C::kColS1 : C::kColS0);
+      const int c = __ldg(cols + j);
+      const bool bad = c < 0 || c >= p.nkb;
+      if (bad && tid == 0) atomicOr(p.status, kDevErrBounds);
+      int kvalid = bad ? 0 : p.N - c * BK;
+      if (kvalid > BK) kvalid = BK;
+      if (!mbar_wait(&bar->s_full[sb], (j >> 1) & 1, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[BK];
+#pragma unroll
+      for (int ch = 0; ch < BK / 32; ++ch)
+        tmem_ld_32x32b_x32(s_col + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
+      tmem_ld_wait();
+      reg_fence(sr);
+
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BK; ++i) {
+        const float x = i < kvalid ? u2f(sr[i]) : -INFINITY;
+        mx = fmaxf(mx, x);
+      }
+      const float m_tile = mx * p.scale_log2;
+      const bool rebase = m_tile > m + kRebaseLog2;
+      const float m_new = rebase ? m_tile : m;
+      const float alpha = rebase ? fast_exp2(m - m_new) : 1.0f;  // exp2(-inf) = 0
+      const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+
+      float sum = 0.0f;
+#pragma unroll
+      for (int ch = 0; ch < BK / 32; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c0 = ch * 32 + 2 * i;
+          const float p0 =
+              c0 < kvalid ? fast_exp2(fmaf(u2f(sr[c0]), p.scale_log2, -m_use)) : 0.0f;
+          const float p1 =
+              c0 + 1 < kvalid ? fast_exp2(fmaf(u2f(sr[c0 + 1]), p.scale_log2, -m_use)) : 0.0f;
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_32x32b_x16(s_col + ch * 16, pk);
+      }
+      l = l * alpha + sum;
+      m = m_new;
+      tmem_st_wait();
+
+      // Re-base O (PV_{j-1} must have landed) when any row of this warp moved.
+      if (j > 0 && __any_sync(0xffffffffu, rebase)) {
+        if (!mbar_wait(&bar->o_full, (j - 1) & 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(lane_base + C::kColO + ch * 32, o);
+          tmem_ld_wait();
+          reg_fence(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * alpha);
+          tmem_st_32x32b_x32(lane_base + C::kColO + ch * 32, o);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->p_full[sb]);
+    }
+
+    // ---- epilogue: O / l -> bf16, lse
+    if (ok && n > 0) ok = mbar_wait(&bar->o_final, 0, abort_flag, p.status);
+    tc_fence_after();
+    svg_bf16* out = p.out[sel] + (static_cast<size_t>(bh) * p.N + row) * D;
+    const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+    const bool have_o = ok && n > 0;
+#pragma unroll
+    for (int ch = 0; ch < D / 32; ++ch) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld_32x32b_x32(lane_base + C::kColO + ch * 32, o);
+        tmem_ld_wait();
+        reg_fence(o);
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        pk[i] = have_o ? pack_bf16x2(u2f(o[2 * i]) * inv_l, u2f(o[2 * i + 1]) * inv_l) : 0u;
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + ch * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+    }
+    if (p.lse != nullptr && row_valid) {
+      p.lse[static_cast<size_t>(bh) * p.N + row] =
+          (have_o && l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, int BK>
+cudaError_t launch_impl(const Dims& d, const AttnParams& p, cudaStream_t stream) {
+  using C = Cfg<D, BK>;
+  auto kern = sparse_attention_kernel<D, BK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(d.nqb, d.BH);
+  kern<<<grid, kThreads, C::kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* status,
+                                    cudaStream_t stream) {
+  AttnParams p;
+  memset(&p, 0, sizeof(p));
+  const bool perm = a.qp != nullptr;
+  if (!make_tmap_bf16(&p.tm_q[0], a.q, d.d, d.N, d.BH, d.bq) ||
+      !make_tmap_bf16(&p.tm_k[0], a.k, d.d, d.N, d.BH, d.bk) ||
+      !make_tmap_bf16(&p.tm_v[0], a.v, d.d, d.N, d.BH, d.bk))
+    return cudaErrorInvalidValue;
+  if (perm) {
+    if (!make_tmap_bf16(&p.tm_q[1], a.qp, d.d, d.N, d.BH, d.bq) ||
+        !make_tmap_bf16(&p.tm_k[1], a.kp, d.d, d.N, d.BH, d.bk) ||
+        !make_tmap_bf16(&p.tm_v[1], a.vp, d.d, d.N, d.BH, d.bk))
+      return cudaErrorInvalidValue;
+  } else {
+    p.tm_q[1] = p.tm_q[0];
+    p.tm_k[1] = p.tm_k[0];
+    p.tm_v[1] = p.tm_v[0];
+  }
+  p.labels = a.labels;
+  p.row_ptr[0] = a.row_ptr_s;
+  p.col_idx[0] = a.col_idx_s;
+  p.row_ptr[1] = a.row_ptr_t ? a.row_ptr_t : a.row_ptr_s;
+  p.col_idx[1] = a.col_idx_t ? a.col_idx_t : a.col_idx_s;
+  p.out[0] = a.o;
+  p.out[1] = a.op ? a.op : a.o;
+  p.lse = a.lse;
+  p.status = status;
+  p.N = d.N;
+  p.BH = d.BH;
+  p.nqb = d.nqb;
+  p.nkb = d.nkb;
+  p.bq = d.bq;
+  p.bk = d.bk;
+  p.has_permuted = perm && a.op != nullptr && a.row_ptr_t != nullptr && a.col_idx_t != nullptr;
+  p.scale_log2 = d.scale * 1.4426950408889634f;
+  if (d.d == 128 && d.bk == 128) return launch_impl<128, 128>(d, p, stream);
+  if (d.d == 128 && d.bk == 64) return launch_impl<128, 64>(d, p, stream);
+  if (d.d == 64 && d.bk == 128) return launch_impl<64, 128>(d, p, stream);
+  return launch_impl<64, 64>(d, p, stream);
+}
+
+}  // namespace svg

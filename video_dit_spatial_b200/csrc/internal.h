@@ -1,0 +1,120 @@
+// Host-side declarations shared by the translation units of libsvg.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "svg.h"
+
+namespace svg {
+
+// Derived sizes of a validated geometry.
+struct Dims {
+  int32_t B, H, BH, T, P, n_text, d, bq, bk, s, w;
+  int32_t N, Nv, nqb, nkb;
+  float scale;
+};
+
+Dims make_dims(const svg_geom& g);
+
+// Closed-form CSR row of a block mask: the key blocks of row r are the run
+// [c_lo, c_hi] (empty when c_lo > c_hi) followed by the run [t_lo, t_hi]
+// (empty when t_lo > t_hi), the second starting after the first. Shared by the
+// host nnz count and the device builder so both agree by construction.
+struct MaskRow {
+  int32_t c_lo, c_hi, t_lo, t_hi;
+  __host__ __device__ int32_t count() const {
+    int32_t n = 0;
+    if (c_hi >= c_lo) n += c_hi - c_lo + 1;
+    if (t_hi >= t_lo) n += t_hi - t_lo + 1;
+    return n;
+  }
+  __host__ __device__ int32_t at(int32_t k) const {
+    const int32_t n1 = (c_hi >= c_lo) ? (c_hi - c_lo + 1) : 0;
+    return k < n1 ? c_lo + k : t_lo + (k - n1);
+  }
+};
+
+struct MaskGeom {
+  int32_t N, Nv, bq, bk, nkb;
+  int32_t group;   // tokens per group in the layout: P (spatial), T (temporal)
+  int32_t ngroups; // number of groups: T (spatial), P (temporal)
+  int32_t band;    // s (spatial) or w (temporal)
+  int32_t dense;   // 1: every block is on
+};
+
+__host__ __device__ inline MaskRow mask_row(const MaskGeom& m, int32_t r) {
+  MaskRow out;
+  const int32_t lo = r * m.bq;
+  const int32_t hi = (lo + m.bq < m.N) ? lo + m.bq : m.N;  // exclusive
+  const bool row_text = hi > m.Nv;
+  const int32_t text_first = m.Nv / m.bk;  // key block holding the first text token
+  if (m.dense || row_text) {
+    out.c_lo = 0;
+    out.c_hi = m.nkb - 1;
+    out.t_lo = 1;
+    out.t_hi = 0;
+    return out;
+  }
+  // Video-only query block: its groups form the interval [g_lo, g_hi].
+  const int32_t g_lo = lo / m.group;
+  const int32_t g_hi = (hi - 1) / m.group;
+  const int32_t a = (g_lo - m.band > 0) ? g_lo - m.band : 0;
+  const int64_t z64 = static_cast<int64_t>(g_hi) + m.band;
+  const int32_t z = (z64 < m.ngroups - 1) ? static_cast<int32_t>(z64) : m.ngroups - 1;
+  const int64_t first_key = static_cast<int64_t>(a) * m.group;
+  int64_t last_key = static_cast<int64_t>(z + 1) * m.group - 1;
+  if (last_key > m.Nv - 1) last_key = m.Nv - 1;
+  out.c_lo = static_cast<int32_t>(first_key / m.bk);
+  out.c_hi = static_cast<int32_t>(last_key / m.bk);
+  if (m.N > m.Nv) {
+    out.t_lo = (text_first > out.c_hi) ? text_first : out.c_hi + 1;
+    out.t_hi = m.nkb - 1;
+  } else {
+    out.t_lo = 1;
+    out.t_hi = 0;
+  }
+  return out;
+}
+
+MaskGeom make_mask_geom(const Dims& d, int32_t kind);
+
+// Device address of this module's status word on the current device.
+int* device_status_word(cudaError_t* err);
+
+// Tensor map of a [BH, N, d] bf16 tensor with a (64 x rows x 1) box, 128-byte swizzle.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int32_t d, int32_t N, int32_t BH,
+                    int32_t box_rows);
+
+// Launchers (validated arguments; return the launch error).
+cudaError_t launch_permute(const Dims& d, int n_tensors, const svg_bf16* const* in,
+                           svg_bf16* const* out, const int8_t* labels, bool inverse,
+                           cudaStream_t stream);
+cudaError_t launch_block_mask(const Dims& d, int32_t kind, int32_t* row_ptr, int32_t* col_idx,
+                              cudaStream_t stream);
+
+struct AttnArgs {
+  const svg_bf16 *q, *k, *v, *qp, *kp, *vp;
+  const int8_t* labels;
+  const int32_t *row_ptr_s, *col_idx_s, *row_ptr_t, *col_idx_t;
+  svg_bf16 *o, *op;
+  float* lse;
+};
+cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* status,
+                                    cudaStream_t stream);
+
+struct ProfileArgs {
+  const svg_bf16 *q, *k, *v;
+  const int32_t* sample_idx;
+  int32_t n_samples;
+  int8_t* labels;
+  float* mse;
+  float* partial;  // [BH][2][n_tiles]
+};
+int32_t profile_tiles(int32_t n_samples);
+cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cudaStream_t stream);
+
+cudaError_t launch_wait_selftest(long long limit_cycles, int* status, cudaStream_t stream);
+
+}  // namespace svg

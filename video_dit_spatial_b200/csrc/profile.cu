@@ -1,0 +1,473 @@
+// Online profiling of Sparse VideoGen (arXiv 2502.01776 abstract: "an online
+// profiling strategy to capture the dynamic sparse patterns and predict the
+// type of attention head"). For sampled query rows of every head, full
+// attention is compared with spatial-masked and temporal-masked attention by
+// the mean squared error of the outputs; the mask with the smaller error names
+// the head's type.
+//
+// One CTA = one (b*H + h, mask X in {spatial, temporal}, tile of 128 sampled
+// rows). It runs flash attention of its 128 gathered query rows over ALL keys
+// (128-key tiles, TMA-fed), keeping two online softmaxes side by side: the
+// full one and the token-level masked one. Tensor memory: S double buffer
+// (columns 0 and 128), O_full (256), O_X (256 + d); P_full and P_X (bf16)
+// overwrite the two halves of their S buffer. The masked product P_X V is
+// skipped for key tiles where no row of the CTA has an allowed key. Each CTA
+// then reduces sum((O_X - O_full)^2) over its rows in a fixed order into the
+// workspace; a second kernel adds the tiles in a fixed order and labels the
+// head. The full-attention half is computed identically by both mask CTAs.
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace svg {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kTile = 128;  // sampled rows per CTA and keys per tile
+constexpr float kRebaseLog2 = 8.0f;
+
+template <int D>
+struct PCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kPanel = 128 * 128;  // 128 rows x 128 B
+  static constexpr int kQBytes = kPanels * kPanel;
+  static constexpr int kKVBytes = kPanels * kPanel;
+  static constexpr int kStages = D == 128 ? 2 : 3;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kBarBytes = 1024;
+  static constexpr int kUsed = kOffBar + kBarBytes + 1024;
+  static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColOF = 256, kColOX = 256 + D;
+};
+
+struct __align__(64) ProfParams {
+  CUtensorMap tm_k, tm_v;
+  const svg_bf16* q;
+  const int32_t* sample_idx;
+  float* partial;  // [BH][2][n_tiles]
+  int* status;
+  int32_t n_samples, n_tiles;
+  int32_t N, Nv, T, P, s, w, nkt;
+  float scale_log2;
+};
+
+struct PBarriers {
+  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full, o_final, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int x_active[2][4];
+  float red[128];
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ void named_sync_softmax() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_constant__ ProfParams p) {
+  using C = PCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  PBarriers* bar = reinterpret_cast<PBarriers*>(smem + C::kOffBar);
+  volatile int* abort_flag = &bar->abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int tile = blockIdx.x;
+  const int X = blockIdx.y;  // 0: spatial mask, 1: temporal mask
+  const int bh = blockIdx.z;
+  const int n = p.nkt;
+
+  if (warp == 0) {
+    tmem_alloc(&bar->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 32) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->s_full[s], 1);
+      mbar_init(&bar->p_full[s], 128);
+    }
+    mbar_init(&bar->o_full, 1);
+    mbar_init(&bar->o_final, 1);
+    mbar_init(&bar->drain, 1);
+    bar->abort_flag = 0;
+    fence_mbar_init();
+  }
+  // Gather the sampled Q rows into the swizzled K-major tile (rows past the
+  // sample count, and out-of-range indices, become zero rows).
+  int qrow = -1;
+  if (tid < 128) {
+    const int si = tile * kTile + tid;
+    if (si < p.n_samples) {
+      const int r = __ldg(p.sample_idx + si);
+      if (r >= 0 && r < p.Nv) {
+        qrow = r;
+      } else {
+        atomicOr(p.status, kDevErrBounds);
+      }
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(
+        p.q + (static_cast<size_t>(bh) * p.N + (qrow >= 0 ? qrow : 0)) * D);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 v = qrow >= 0 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      const int pn = c >> 3, cc = c & 7;
+      *reinterpret_cast<uint4*>(sQ + pn * C::kPanel + tid * 128 + ((cc ^ (tid & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == kProducerWarp) {
+    if (lane_id() == 0) {
+      const uint64_t keep = l2_policy_evict_last();
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % C::kStages;
+        if (!mbar_wait(&bar->kv_empty[st], ((j / C::kStages) & 1) ^ 1, abort_flag, p.status))
+          break;
+        mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kPanel, &p.tm_k, &bar->k_full[st],
+                           pn * 64, j * kTile, bh, keep);
+        mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kPanel, &p.tm_v, &bar->v_full[st],
+                           pn * 64, j * kTile, bh, keep);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
+          const int st = j % C::kStages;
+          const uint32_t par = (j / C::kStages) & 1;
+          long long t0 = clock64();
+          while (!(mbar_try_wait(&bar->k_full[st], par) && mbar_try_wait(&bar->v_full[st], par)) &&
+                 clock64() - t0 < kWaitLimitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane_id() == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTile, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t k_addr = smem_u32(sK);
+      const uint32_t v_addr = smem_u32(sV);
+      bool x_started = false;
+      for (int j = 0; j <= n; ++j) {
+        if (j < n) {
+          const int st = j % C::kStages;
+          const uint32_t s_col = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
+          if (!mbar_wait(&bar->k_full[st], (j / C::kStages) & 1, abort_flag, p.status)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kPanel + (kk & 3) * 32;
+            mma_bf16_ss(s_col, sdesc_sw128(q_addr + off, 16, 1024),
+                        sdesc_sw128(k_addr + st * C::kKVBytes + off, 16, 1024), idesc_qk,
+                        kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bar->s_full[j & 1]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int st = jj % C::kStages;
+          const int sb = jj & 1;
+          const uint32_t p_col = tmem + (sb ? C::kColS1 : C::kColS0);
+          if (!mbar_wait(&bar->p_full[sb], (jj >> 1) & 1, abort_flag, p.status)) break;
+          if (!mbar_wait(&bar->v_full[st], (jj / C::kStages) & 1, abort_flag, p.status)) break;
+          tc_fence_after();
+          const volatile int* xa = bar->x_active[sb];
+          const bool x_on = (xa[0] | xa[1] | xa[2] | xa[3]) != 0;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t b = sdesc_sw128(v_addr + st * C::kKVBytes + kk * 16 * 128, C::kPanel,
+                                           1024);
+            mma_bf16_ts(tmem + C::kColOF, p_col + kk * 8, b, idesc_pv,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (x_on) {
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t b = sdesc_sw128(v_addr + st * C::kKVBytes + kk * 16 * 128,
+                                             C::kPanel, 1024);
+              mma_bf16_ts(tmem + C::kColOX, p_col + 64 + kk * 8, b, idesc_pv,
+                          (x_started || kk > 0) ? 1u : 0u);
+            }
+            x_started = true;
+          }
+          tc_commit(&bar->kv_empty[st]);
+          tc_commit(&bar->o_full);
+          if (jj == n - 1) tc_commit(&bar->o_final);
+        }
+      }
+      if (*abort_flag) {
+        tc_commit(&bar->drain);
+        long long t0 = clock64();
+        while (!mbar_try_wait(&bar->drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const bool row_valid = qrow >= 0;
+    const int qi = row_valid ? qrow : 0;
+    const int f_i = qi / p.P;
+    const int p_i = qi - f_i * p.P;
+    // spatial: allowed video keys are the frames [f_i - s, f_i + s], one index run
+    const long long s_lo = static_cast<long long>(max(f_i - p.s, 0)) * p.P;
+    const long long s_hi = static_cast<long long>(min(static_cast<long long>(f_i) + p.s + 1,
+                                                      static_cast<long long>(p.T))) * p.P;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float mF = -INFINITY, lF = 0.0f, mX = -INFINITY, lX = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int sb = j & 1;
+      const uint32_t s_col = lane_base + (sb ? C::kColS1 : C::kColS0);
+      const int j0 = j * kTile;
+      int kvalid = p.N - j0;
+      if (kvalid > kTile) kvalid = kTile;
+      // allowed-key bits of this row for the 128 keys of the tile
+      uint32_t bits[4] = {0u, 0u, 0u, 0u};
+      if (X == 0) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) {
+          const int jj = j0 + c;
+          const bool in = c < kvalid && (jj >= p.Nv || (jj >= s_lo && jj < s_hi));
+          bits[c >> 5] |= (in ? 1u : 0u) << (c & 31);
+        }
+      } else {
+        int pj = j0 % p.P;
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) {
+          const int jj = j0 + c;
+          const int dp = pj - p_i;
+          const bool in = c < kvalid && (jj >= p.Nv || (dp <= p.w && -dp <= p.w));
+          bits[c >> 5] |= (in ? 1u : 0u) << (c & 31);
+          pj = (pj + 1 == p.P) ? 0 : pj + 1;
+        }
+      }
+      if (!row_valid) bits[0] = bits[1] = bits[2] = bits[3] = 0u;
+      const bool any_x = (bits[0] | bits[1] | bits[2] | bits[3]) != 0u;
+      const int warp_any = __any_sync(0xffffffffu, any_x) ? 1 : 0;
+
+      if (!mbar_wait(&bar->s_full[sb], (j >> 1) & 1, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[kTile];
+#pragma unroll
+      for (int ch = 0; ch < kTile / 32; ++ch)
+        tmem_ld_32x32b_x32(s_col + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
+      tmem_ld_wait();
+      reg_fence(sr);
+
+      float mxF = -INFINITY, mxX = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) {
+        const float x = u2f(sr[c]);
+        if (c < kvalid) mxF = fmaxf(mxF, x);
+        if ((bits[c >> 5] >> (c & 31)) & 1u) mxX = fmaxf(mxX, x);
+      }
+      const float tF = mxF * p.scale_log2, tX = mxX * p.scale_log2;
+      const bool rbF = tF > mF + kRebaseLog2;
+      const bool rbX = tX > mX + kRebaseLog2;
+      const float mF_new = rbF ? tF : mF, mX_new = rbX ? tX : mX;
+      const float aF = rbF ? fast_exp2(mF - mF_new) : 1.0f;
+      const float aX = rbX ? fast_exp2(mX - mX_new) : 1.0f;
+      const float uF = mF_new == -INFINITY ? 0.0f : mF_new;
+      const float uX = mX_new == -INFINITY ? 0.0f : mX_new;
+      float sumF = 0.0f, sumX = 0.0f;
+#pragma unroll
+      for (int ch = 0; ch < kTile / 32; ++ch) {
+        uint32_t pkF[16], pkX[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c0 = ch * 32 + 2 * i;
+          const float x0 = u2f(sr[c0]), x1 = u2f(sr[c0 + 1]);
+          const float f0 = c0 < kvalid ? fast_exp2(fmaf(x0, p.scale_log2, -uF)) : 0.0f;
+          const float f1 = c0 + 1 < kvalid ? fast_exp2(fmaf(x1, p.scale_log2, -uF)) : 0.0f;
+          const bool in0 = (bits[ch] >> (2 * i)) & 1u;
+          const bool in1 = (bits[ch] >> (2 * i + 1)) & 1u;
+          const float g0 = in0 ? fast_exp2(fmaf(x0, p.scale_log2, -uX)) : 0.0f;
+          const float g1 = in1 ? fast_exp2(fmaf(x1, p.scale_log2, -uX)) : 0.0f;
+          sumF += f0 + f1;
+          sumX += g0 + g1;
+          pkF[i] = pack_bf16x2(f0, f1);
+          pkX[i] = pack_bf16x2(g0, g1);
+        }
+        tmem_st_32x32b_x16(s_col + ch * 16, pkF);
+        tmem_st_32x32b_x16(s_col + 64 + ch * 16, pkX);
+      }
+      lF = lF * aF + sumF;
+      lX = lX * aX + sumX;
+      mF = mF_new;
+      mX = mX_new;
+      tmem_st_wait();
+      if (lane_id() == 0) bar->x_active[sb][warp] = warp_any;
+
+      const bool wF = __any_sync(0xffffffffu, rbF);
+      const bool wX = __any_sync(0xffffffffu, rbX);
+      if (j > 0 && (wF || wX)) {
+        if (!mbar_wait(&bar->o_full, (j - 1) & 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (wF) {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(lane_base + C::kColOF + ch * 32, o);
+            tmem_ld_wait();
+            reg_fence(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * aF);
+            tmem_st_32x32b_x32(lane_base + C::kColOF + ch * 32, o);
+          }
+        }
+        if (wX) {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(lane_base + C::kColOX + ch * 32, o);
+            tmem_ld_wait();
+            reg_fence(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * aX);
+            tmem_st_32x32b_x32(lane_base + C::kColOX + ch * 32, o);
+          }
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->p_full[sb]);
+    }
+
+    // ---- per-row squared error, then a fixed-order CTA sum
+    if (ok && n > 0) ok = mbar_wait(&bar->o_final, 0, abort_flag, p.status);
+    tc_fence_after();
+    float err = 0.0f;
+    if (ok && n > 0) {
+      const float iF = lF > 0.0f ? 1.0f / lF : 0.0f;
+      const float iX = lX > 0.0f ? 1.0f / lX : 0.0f;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t oF[32], oX[32];
+        tmem_ld_32x32b_x32(lane_base + C::kColOF + ch * 32, oF);
+        tmem_ld_32x32b_x32(lane_base + C::kColOX + ch * 32, oX);
+        tmem_ld_wait();
+        reg_fence(oF);
+        reg_fence(oX);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float dlt = u2f(oX[i]) * iX - u2f(oF[i]) * iF;
+          err = fmaf(dlt, dlt, err);
+        }
+      }
+    }
+    bar->red[tid] = row_valid ? err : 0.0f;
+    named_sync_softmax();
+    if (tid == 0) {
+      float acc = 0.0f;
+      for (int i = 0; i < 128; ++i) acc += bar->red[i];
+      p.partial[(static_cast<size_t>(bh) * 2 + X) * p.n_tiles + tile] = ok ? acc : __int_as_float(0x7fc00000);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Sums the per-tile partial errors of each head in tile order and labels it.
+__global__ void profile_finalize_kernel(const float* __restrict__ partial, int32_t BH,
+                                        int32_t n_tiles, float inv_count,
+                                        int8_t* __restrict__ labels, float* __restrict__ mse) {
+  const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+  if (bh >= BH) return;
+  float e[2];
+  for (int x = 0; x < 2; ++x) {
+    const float* src = partial + (static_cast<size_t>(bh) * 2 + x) * n_tiles;
+    float acc = 0.0f;
+    for (int t = 0; t < n_tiles; ++t) acc += src[t];
+    e[x] = acc * inv_count;
+  }
+  labels[bh] = e[1] < e[0] ? SVG_HEAD_TEMPORAL : SVG_HEAD_SPATIAL;
+  if (mse != nullptr) {
+    mse[2 * bh] = e[0];
+    mse[2 * bh + 1] = e[1];
+  }
+}
+
+template <int D>
+cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, float* mse,
+                        cudaStream_t stream) {
+  using C = PCfg<D>;
+  auto kern = profile_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(pp.n_tiles, 2, d.BH), kThreads, C::kSmem, stream>>>(pp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const float inv = 1.0f / (static_cast<float>(pp.n_samples) * static_cast<float>(D));
+  profile_finalize_kernel<<<(d.BH + 127) / 128, 128, 0, stream>>>(pp.partial, d.BH, pp.n_tiles,
+                                                                  inv, labels, mse);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int32_t profile_tiles(int32_t n_samples) { return (n_samples + kTile - 1) / kTile; }
+
+cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cudaStream_t stream) {
+  ProfParams pp;
+  memset(&pp, 0, sizeof(pp));
+  if (!make_tmap_bf16(&pp.tm_k, a.k, d.d, d.N, d.BH, kTile) ||
+      !make_tmap_bf16(&pp.tm_v, a.v, d.d, d.N, d.BH, kTile))
+    return cudaErrorInvalidValue;
+  pp.q = a.q;
+  pp.sample_idx = a.sample_idx;
+  pp.partial = a.partial;
+  pp.status = status;
+  pp.n_samples = a.n_samples;
+  pp.n_tiles = profile_tiles(a.n_samples);
+  pp.N = d.N;
+  pp.Nv = d.Nv;
+  pp.T = d.T;
+  pp.P = d.P;
+  pp.s = d.s;
+  pp.w = d.w;
+  pp.nkt = (d.N + kTile - 1) / kTile;
+  pp.scale_log2 = d.scale * 1.4426950408889634f;
+  if (d.d == 128) return launch_impl<128>(d, pp, a.labels, a.mse, stream);
+  return launch_impl<64>(d, pp, a.labels, a.mse, stream);
+}
+
+}  // namespace svg
