@@ -346,13 +346,17 @@ def layer_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, label: int, T: int, 
         rows = np.arange(N)
     rows = np.asarray(rows, dtype=np.int64)
     kind = MASK_TEMPORAL if label == HEAD_TEMPORAL else MASK_SPATIAL
+    pi = permutation(T, P, n_text) if kind == MASK_TEMPORAL else None
+    layout_rows = rows if pi is None else pi[rows]
     if bm is None:
-        bm = block_mask(kind, T, P, n_text, s, w, block_q, block_k)
+        # Only the block-mask rows the requested query rows fall in are needed.
+        needed = np.unique(layout_rows // block_q)
+        bm = np.zeros((n_blocks(N, block_q), n_blocks(N, block_k)), dtype=bool)
+        bm[needed] = block_mask_rows(kind, needed, T, P, n_text, s, w, block_q, block_k)
     if kind == MASK_SPATIAL:
-        return sparse_attention_rows(q, k, v, bm, block_q, block_k, scale, rows)
-    pi = permutation(T, P, n_text)
+        return sparse_attention_rows(q, k, v, bm, block_q, block_k, scale, layout_rows)
     qp, kp, vp = (permute(x, T, P, n_text) for x in (q, k, v))
-    return sparse_attention_rows(qp, kp, vp, bm, block_q, block_k, scale, pi[rows])
+    return sparse_attention_rows(qp, kp, vp, bm, block_q, block_k, scale, layout_rows)
 
 
 def flops_computed_blocks(bm: np.ndarray, N: int, block_q: int, block_k: int, d: int) -> int:

@@ -19,16 +19,28 @@ def rand_bf16(shape, seed, scale=1.0):
     return (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16)
 
 
-def edge_rows(N, Nv, bq, n_random, seed):
+def edge_rows(N, Nv, bq, n_random, seed, n_blocks=6, layout_to_frame_major=None):
     """Rows every parity check covers: both ends, the video/text boundary, the last
-    query block's first and last row, plus seeded random rows."""
+    query block's first and last row, plus seeded random rows drawn from a few
+    seeded random query blocks (the oracle's cost grows with distinct blocks).
+
+    Rows are chosen in the head's layout; `layout_to_frame_major` (an index
+    array) maps them back to frame-major rows for position-major heads."""
     last_blk = ((N - 1) // bq) * bq
     rows = {0, 1, Nv - 1, N - 1, last_blk, min(last_blk + bq - 1, N - 1)}
     if Nv < N:
         rows.add(Nv)
     rng = np.random.default_rng(seed)
-    rows.update(rng.choice(N, size=min(n_random, N), replace=False).tolist())
-    return np.array(sorted(r for r in rows if 0 <= r < N), dtype=np.int64)
+    nqb = -(-N // bq)
+    blocks = rng.choice(nqb, size=min(n_blocks, nqb), replace=False)
+    per = max(1, n_random // len(blocks))
+    for b in blocks:
+        lo, hi = b * bq, min(N, (b + 1) * bq)
+        rows.update(rng.choice(np.arange(lo, hi), size=min(per, hi - lo), replace=False).tolist())
+    out = np.array(sorted(r for r in rows if 0 <= r < N), dtype=np.int64)
+    if layout_to_frame_major is not None:
+        out = np.sort(layout_to_frame_major[out])
+    return out
 
 
 def assert_close(got: np.ndarray, want: np.ndarray, what: str):

@@ -144,9 +144,11 @@ def test_sparse_attention_full_size_sampled_rows(svg, wl):
     del qd, kd, vd
     sp = [h for h in range(wl.H) if kinds[h] == 0][:2]
     tp = [h for h in range(wl.H) if kinds[h] == 1][:2]
-    rows = edge_rows(wl.N, wl.N_v, wl.block_q, 40, seed=11)
+    inv_pi = O.inverse_permutation(O.permutation(wl.T, wl.P, wl.n_text))
     for b in range(wl.B):
         for h in sp + tp:
+            rows = edge_rows(wl.N, wl.N_v, wl.block_q, 40, seed=11 + h,
+                             layout_to_frame_major=inv_pi if kinds[h] == 1 else None)
             qn, kn, vn = to_f64(q[b, h]), to_f64(k[b, h]), to_f64(v[b, h])
             want, _ = O.layer_rows(qn, kn, vn, kinds[h], wl.T, wl.P, wl.n_text, wl.spatial_band,
                                    wl.temporal_width, wl.block_q, wl.block_k, wl.scale, rows=rows)
