@@ -30,6 +30,15 @@ constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr float kRebaseLog2 = 8.0f;  // lazy re-basing threshold (log2 units)
 
+struct Barriers {
+  uint64_t q_full;
+  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full, o_final, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
 template <int D, int BK>
 struct Cfg {
   static constexpr int kPanels = D / 64;            // 128-byte wide column panels
@@ -42,12 +51,14 @@ struct Cfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
   static constexpr int kOffBar = kOffV + kStages * kKVBytes;
-  static constexpr int kBarBytes = 256;
+  static constexpr int kBarBytes = (static_cast<int>(sizeof(Barriers)) + 127) / 128 * 128;
   static constexpr int kUsed = kOffBar + kBarBytes + 1024;  // + alignment slack
   // Keep one CTA per SM: each CTA takes all 512 tensor-memory columns.
   static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+  static_assert(kOffBar + kBarBytes + 1024 <= kSmem, "bookkeeping must fit the allocation");
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
 
 struct __align__(64) AttnParams {
@@ -63,14 +74,6 @@ struct __align__(64) AttnParams {
   float scale_log2;
 };
 
-struct Barriers {
-  uint64_t q_full;
-  uint64_t k_full[3], v_full[3], kv_empty[3];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_full, o_final, drain;
-  uint32_t tmem_base;
-  int abort_flag;
-};
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
@@ -361,6 +364,432 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ===========================================================================
+// Paired-tile variant (block_q = 128): one CTA = two consecutive query blocks
+// A = 2p and B = 2p+1 of one head. The K/V tiles of the union of the two CSR
+// rows stream once through separate K and V rings and serve both tiles.
+// 384 threads (three warpgroups): warps 0-3 softmax of tile A, warps 4-7
+// softmax of tile B, warp 8 TMA producer, warp 9 MMA issuer, warps 10-11 idle.
+// The kernel launches at 168 registers per thread (three warps per SM
+// sub-partition); the producer warpgroup then gives registers back
+// (setmaxnreg.dec to 56) and the softmax warpgroups take them (setmaxnreg.inc
+// to 224): 224 + 224 + 56 = 3 x 168 per sub-partition. Tensor memory: S_A 0, O_A 128,
+// S_B 256, O_B 384 (P_t overwrites the first half of S_t). Per union step u
+// the MMA issue order is PV_A(u-1), QK_A(u), PV_B(u-1), QK_B(u): each tile's
+// softmax overlaps the other tile's PV and QK, every PV is issued at most one
+// step after its block, and PV_t(j-1) always precedes QK_t(j), so the commit of
+// S_t(j) also retires PV_t(j-1) (the softmax may then re-base O_t freely).
+// ===========================================================================
+constexpr int kPairThreads = 384;
+constexpr int kPairProducerWarp = 8;
+constexpr int kPairMmaWarp = 9;
+constexpr int kPairLaunchRegs = 168;   // per thread at launch (3 warps per sub-partition)
+constexpr int kPairSoftmaxRegs = 224;  // softmax warpgroups after setmaxnreg.inc
+constexpr int kPairOtherRegs = 56;     // producer / MMA warpgroup after setmaxnreg.dec
+static_assert(2 * kPairSoftmaxRegs + kPairOtherRegs == 3 * kPairLaunchRegs,
+              "register split must equal the launch allocation");
+
+struct PairBarriers {
+  uint64_t q_full;
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t s_full[2], p_full[2], o_final[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D, int BK>
+struct PairCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kQPanel = 128 * 128;
+  static constexpr int kKVPanel = BK * 128;
+  static constexpr int kQBytes = kPanels * kQPanel;     // one query tile
+  static constexpr int kKVBytes = kPanels * kKVPanel;   // one K (or V) tile
+  static constexpr int kStages = (D == 128 && BK == 128) ? 2 : 3;
+  static constexpr int kOffQ = 0;                        // Q_A, then Q_B
+  static constexpr int kOffK = kOffQ + 2 * kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kBarBytes = (static_cast<int>(sizeof(PairBarriers)) + 127) / 128 * 128;
+  static constexpr int kUsed = kOffBar + kBarBytes + 1024;
+  static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  // tensor-memory columns of tile t's S (P) and O
+  static __device__ __forceinline__ uint32_t col_s(int t) { return t ? 256u : 0u; }
+  static __device__ __forceinline__ uint32_t col_o(int t) { return t ? 384u : 128u; }
+  static_assert(kOffBar + kBarBytes + 1024 <= kSmem, "bookkeeping must fit the allocation");
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+};
+
+
+// Walks the ascending union of two CSR rows, one block per call.
+struct UnionWalk {
+  const int32_t* a;
+  const int32_t* b;
+  int na, nb, ia = 0, ib = 0;
+  __device__ __forceinline__ int next(bool& in_a, bool& in_b) {
+    const int ca = ia < na ? __ldg(a + ia) : 0x7fffffff;
+    const int cb = ib < nb ? __ldg(b + ib) : 0x7fffffff;
+    const int c = ca < cb ? ca : cb;
+    in_a = ca == c && ia < na;
+    in_b = cb == c && ib < nb;
+    ia += in_a;
+    ib += in_b;
+    return c;
+  }
+};
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    sparse_attention_pair_kernel(const __grid_constant__ AttnParams p) {
+  using C = PairCfg<D, BK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  PairBarriers* bar = reinterpret_cast<PairBarriers*>(smem + C::kOffBar);
+  volatile int* abort_flag = &bar->abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int npairs = (p.nqb + 1) >> 1;
+  const int pair = npairs - 1 - static_cast<int>(blockIdx.x);  // text-heavy rows first
+  const int bh = blockIdx.y;
+
+  const int label = p.labels ? static_cast<int>(p.labels[bh]) : SVG_HEAD_SPATIAL;
+  const int sel = label == SVG_HEAD_TEMPORAL ? 1 : 0;
+  if ((label != SVG_HEAD_SPATIAL && label != SVG_HEAD_TEMPORAL) || (sel == 1 && !p.has_permuted)) {
+    if (tid == 0) atomicOr(p.status, kDevErrBounds);
+    return;
+  }
+  // CSR rows of the two tiles (tile B may not exist at an odd tail)
+  int qb[2], nt[2];
+  const int32_t* cols[2];
+  for (int t = 0; t < 2; ++t) {
+    qb[t] = 2 * pair + t;
+    nt[t] = 0;
+    cols[t] = p.col_idx[sel];
+    if (qb[t] < p.nqb) {
+      const int32_t r0 = __ldg(p.row_ptr[sel] + qb[t]);
+      int32_t len = __ldg(p.row_ptr[sel] + qb[t] + 1) - r0;
+      if (len < 0 || len > p.nkb) {
+        if (tid == 0) atomicOr(p.status, kDevErrBounds);
+        len = 0;
+      }
+      nt[t] = len;
+      cols[t] = p.col_idx[sel] + r0;
+    }
+  }
+
+  if (warp == 0) {
+    tmem_alloc(&bar->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 32) {
+    mbar_init(&bar->q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_empty[s], 1);
+      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->v_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar->s_full[t], 1);
+      mbar_init(&bar->p_full[t], 128);
+      mbar_init(&bar->o_final[t], 1);
+    }
+    mbar_init(&bar->drain, 1);
+    bar->abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+  const bool any_work = nt[0] > 0 || nt[1] > 0;
+
+  if (warp >= 8) {
+    // producer / MMA warpgroup: hand registers to the softmax warpgroups
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairOtherRegs));
+    if (warp == kPairProducerWarp) {
+      // ------------------------------------------------------------ producer
+      if (lane_id() == 0 && any_work) {
+        const CUtensorMap* mq = &p.tm_q[sel];
+        const CUtensorMap* mk = &p.tm_k[sel];
+        const CUtensorMap* mv = &p.tm_v[sel];
+        const uint64_t keep = l2_policy_evict_last();
+        uint32_t qbytes = 0;
+        for (int t = 0; t < 2; ++t) qbytes += nt[t] > 0 ? C::kQBytes : 0;
+        mbar_arrive_expect_tx(&bar->q_full, qbytes);
+        for (int t = 0; t < 2; ++t)
+          if (nt[t] > 0)
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d(sQ + t * C::kQBytes + pn * C::kQPanel, mq, &bar->q_full, pn * 64,
+                          qb[t] * 128, bh);
+        UnionWalk walk{cols[0], cols[1], nt[0], nt[1]};
+        int issued = 0;
+        for (int u = 0;; ++u) {
+          bool ia, ib;
+          int c = walk.next(ia, ib);
+          if (!ia && !ib) break;
+          if (c < 0 || c >= p.nkb) c = 0;  // flagged and masked by the softmax warps
+          const int st = u % C::kStages;
+          const uint32_t par = ((u / C::kStages) & 1) ^ 1;
+          if (!mbar_wait(&bar->k_empty[st], par, abort_flag, p.status)) break;
+          mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kKVPanel, mk, &bar->k_full[st],
+                             pn * 64, c * BK, bh, keep);
+          if (!mbar_wait(&bar->v_empty[st], par, abort_flag, p.status)) {
+            issued = -(u + 1);  // K of step u is in flight, V is not
+            break;
+          }
+          mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kKVPanel, mv, &bar->v_full[st],
+                             pn * 64, c * BK, bh, keep);
+          issued = u + 1;
+        }
+        if (*abort_flag) {
+          // Let every copy this thread started land before the CTA retires.
+          const int done = issued < 0 ? -issued : issued;
+          for (int u = (done > C::kStages ? done - C::kStages : 0); u < done; ++u) {
+            const int st = u % C::kStages;
+            const uint32_t par = (u / C::kStages) & 1;
+            const bool v_issued = issued >= 0 || u < done - 1;
+            long long t0 = clock64();
+            while (!(mbar_try_wait(&bar->k_full[st], par) &&
+                     (!v_issued || mbar_try_wait(&bar->v_full[st], par))) &&
+                   clock64() - t0 < kWaitLimitCycles) {
+            }
+          }
+        }
+      }
+    } else if (warp == kPairMmaWarp) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane_id() == 0 && any_work) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BK, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        const uint32_t q_addr = smem_u32(sQ);
+        const uint32_t k_addr = smem_u32(sK);
+        const uint32_t v_addr = smem_u32(sV);
+        bool ok = mbar_wait(&bar->q_full, 0, abort_flag, p.status);
+        tc_fence_after();
+        UnionWalk walk{cols[0], cols[1], nt[0], nt[1]};
+        bool prev_in[2] = {false, false};
+        int pv_done[2] = {0, 0};
+        for (int u = 0; ok; ++u) {
+          bool in[2];
+          walk.next(in[0], in[1]);
+          const bool step = in[0] || in[1];  // false: drain step after the last block
+          if (!step && !prev_in[0] && !prev_in[1]) break;
+          const int st = u % C::kStages;
+          const int pst = (u + C::kStages - 1) % C::kStages;
+          bool k_ready = false, v_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (prev_in[t]) {  // PV_t of the previous step
+              if (!v_ready) {
+                ok = mbar_wait(&bar->v_full[pst], ((u - 1) / C::kStages) & 1, abort_flag, p.status);
+                v_ready = true;
+              }
+              if (ok) ok = mbar_wait(&bar->p_full[t], pv_done[t] & 1, abort_flag, p.status);
+              if (!ok) break;
+              tc_fence_after();
+  #pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint64_t b = sdesc_sw128(v_addr + pst * C::kKVBytes + kk * 16 * 128,
+                                               C::kKVPanel, 1024);
+                mma_bf16_ts(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv,
+                            (pv_done[t] > 0 || kk > 0) ? 1u : 0u);
+              }
+              ++pv_done[t];
+              if (pv_done[t] == nt[t]) tc_commit(&bar->o_final[t]);
+            }
+            if (step && in[t]) {  // QK_t of this step
+              if (!k_ready) {
+                ok = mbar_wait(&bar->k_full[st], (u / C::kStages) & 1, abort_flag, p.status);
+                k_ready = true;
+                if (!ok) break;
+              }
+              tc_fence_after();
+  #pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk & 3) * 32;
+                const uint64_t a = sdesc_sw128(q_addr + t * C::kQBytes + (kk >> 2) * C::kQPanel + off,
+                                               16, 1024);
+                const uint64_t b = sdesc_sw128(
+                    k_addr + st * C::kKVBytes + (kk >> 2) * C::kKVPanel + off, 16, 1024);
+                mma_bf16_ss(tmem + C::col_s(t), a, b, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(&bar->s_full[t]);
+            }
+          }
+          if (!ok) break;
+          if (u >= 1) tc_commit(&bar->v_empty[pst]);
+          if (step) tc_commit(&bar->k_empty[st]);
+          prev_in[0] = in[0];
+          prev_in[1] = in[1];
+          if (!step) break;
+        }
+        if (*abort_flag) {
+          tc_commit(&bar->drain);
+          long long t0 = clock64();
+          while (!mbar_try_wait(&bar->drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+          }
+        }
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPairSoftmaxRegs));
+    // ------------------------------------------------------------ softmax (tile t)
+    const int t = warp >> 2;
+    const int r = tid & 127;  // row within the tile = TMEM lane
+    const int row = qb[t] * 128 + r;
+    const bool row_valid = qb[t] < p.nqb && row < p.N;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_col = lane_base + C::col_s(t);
+    const uint32_t o_col = lane_base + C::col_o(t);
+    const int n = nt[t];
+    const int32_t* my_cols = cols[t];
+    float m = -INFINITY;  // running base, log2 units
+    float l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int c = __ldg(my_cols + j);
+      const bool bad = c < 0 || c >= p.nkb;
+      if (bad && r == 0) atomicOr(p.status, kDevErrBounds);
+      int kvalid = bad ? 0 : p.N - c * BK;
+      if (kvalid > BK) kvalid = BK;
+      if (!mbar_wait(&bar->s_full[t], j & 1, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[BK];
+#pragma unroll
+      for (int ch = 0; ch < BK / 32; ++ch)
+        tmem_ld_32x32b_x32(s_col + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
+      tmem_ld_wait();
+      reg_fence(sr);
+      if (kvalid < BK) {  // the ragged last key block (or a flagged index)
+#pragma unroll
+        for (int i = 0; i < BK; ++i)
+          if (i >= kvalid) sr[i] = __float_as_uint(-INFINITY);
+      }
+      float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BK; i += 8) {
+        x0 = fmax3(x0, u2f(sr[i]), u2f(sr[i + 1]));
+        x1 = fmax3(x1, u2f(sr[i + 2]), u2f(sr[i + 3]));
+        x2 = fmax3(x2, u2f(sr[i + 4]), u2f(sr[i + 5]));
+        x3 = fmax3(x3, u2f(sr[i + 6]), u2f(sr[i + 7]));
+      }
+      const float m_tile = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)) * p.scale_log2;
+      const bool rebase = m_tile > m + kRebaseLog2;
+      const float m_new = rebase ? m_tile : m;
+      const float alpha = rebase ? fast_exp2(m - m_new) : 1.0f;  // exp2(-inf) = 0
+      const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+      float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+      for (int ch = 0; ch < BK / 32; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c0 = ch * 32 + 2 * i;
+          float y0, y1;
+          ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -m_use, -m_use);
+          const float e0 = fast_exp2(y0), e1 = fast_exp2(y1);
+          fadd2(s0, s1, s0, s1, e0, e1);
+          pk[i] = pack_bf16x2(e0, e1);
+        }
+        tmem_st_32x32b_x16(s_col + ch * 16, pk);
+      }
+      l = l * alpha + (s0 + s1);
+      m = m_new;
+      tmem_st_wait();
+      // PV_t(j-1) retired with QK_t(j), so O_t may be re-based right away.
+      if (j > 0 && __any_sync(0xffffffffu, rebase)) {
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(o_col + ch * 32, o);
+          tmem_ld_wait();
+          reg_fence(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * alpha);
+          tmem_st_32x32b_x32(o_col + ch * 32, o);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->p_full[t]);
+    }
+
+    // ---- epilogue: O / l -> bf16, lse
+    if (ok && n > 0) ok = mbar_wait(&bar->o_final[t], 0, abort_flag, p.status);
+    tc_fence_after();
+    const bool have_o = __all_sync(0xffffffffu, ok) && n > 0;
+    svg_bf16* out = p.out[sel] + (static_cast<size_t>(bh) * p.N + row) * D;
+    const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+    for (int ch = 0; ch < D / 32; ++ch) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld_32x32b_x32(o_col + ch * 32, o);
+        tmem_ld_wait();
+        reg_fence(o);
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        pk[i] = have_o ? pack_bf16x2(u2f(o[2 * i]) * inv_l, u2f(o[2 * i + 1]) * inv_l) : 0u;
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + ch * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+    }
+    if (p.lse != nullptr && row_valid) {
+      p.lse[static_cast<size_t>(bh) * p.N + row] =
+          (have_o && l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, int BK>
+cudaError_t launch_impl(const Dims& d, const AttnParams& p, cudaStream_t stream);
+
+template <int D, int BK>
+cudaError_t launch_pair(const Dims& d, const AttnParams& p, cudaStream_t stream) {
+  using C = PairCfg<D, BK>;
+  auto kern = sparse_attention_pair_kernel<D, BK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  // The register hand-over inside the kernel is only balanced when the kernel
+  // launches at exactly kPairLaunchRegs per thread; otherwise (or if a CTA
+  // cannot be resident) use the single-tile kernel.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  int resident = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kPairThreads, C::kSmem);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kPairLaunchRegs || resident < 1) return launch_impl<D, BK>(d, p, stream);
+  dim3 grid((d.nqb + 1) / 2, d.BH);
+  kern<<<grid, kPairThreads, C::kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int D, int BK>
 cudaError_t launch_impl(const Dims& d, const AttnParams& p, cudaStream_t stream) {
   using C = Cfg<D, BK>;
@@ -410,6 +839,12 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
   p.bk = d.bk;
   p.has_permuted = perm && a.op != nullptr && a.row_ptr_t != nullptr && a.col_idx_t != nullptr;
   p.scale_log2 = d.scale * 1.4426950408889634f;
+  if (d.bq == 128) {
+    if (d.d == 128 && d.bk == 128) return launch_pair<128, 128>(d, p, stream);
+    if (d.d == 128 && d.bk == 64) return launch_pair<128, 64>(d, p, stream);
+    if (d.d == 64 && d.bk == 128) return launch_pair<64, 128>(d, p, stream);
+    return launch_pair<64, 64>(d, p, stream);
+  }
   if (d.d == 128 && d.bk == 128) return launch_impl<128, 128>(d, p, stream);
   if (d.d == 128 && d.bk == 64) return launch_impl<128, 64>(d, p, stream);
   if (d.d == 64 && d.bk == 128) return launch_impl<64, 128>(d, p, stream);

@@ -8,24 +8,48 @@
 // One CTA = one (b*H + h, mask X in {spatial, temporal}, tile of 128 sampled
 // rows). It runs flash attention of its 128 gathered query rows over ALL keys
 // (128-key tiles, TMA-fed), keeping two online softmaxes side by side: the
-// full one and the token-level masked one. Tensor memory: S double buffer
-// (columns 0 and 128), O_full (256), O_X (256 + d); P_full and P_X (bf16)
-// overwrite the two halves of their S buffer. The masked product P_X V is
-// skipped for key tiles where no row of the CTA has an allowed key. Each CTA
-// then reduces sum((O_X - O_full)^2) over its rows in a fixed order into the
-// workspace; a second kernel adds the tiles in a fixed order and labels the
-// head. The full-attention half is computed identically by both mask CTAs.
+// full one and the token-level masked one, each with its own running maximum.
+//
+// 320 threads: warps 0-7 softmax, warp 8 TMA producer, warp 9 MMA issuer.
+// Warps w and w+4 own the same 32 query rows (TMEM lanes 32*(w%4)..+31) and
+// split each 128-key tile into columns [0,64) and [64,128); they exchange row
+// maxima through shared memory (one 64-thread named barrier per warp pair)
+// and keep partial row sums that are added once at the end.
+// Tensor memory: S double buffer (columns 0 and 128), O_full (256), O_X
+// (256 + d); P_full and P_X (bf16) overwrite the two halves of their S buffer.
+// The allowed keys of a row inside a tile are at most a few index runs
+// (spatial: the frames [f-s, f+s]; temporal: positions [p-w, p+w] of each
+// frame; text keys always), built as bit ranges. P_X = P_full * 2^(mF - mX) on
+// allowed keys; the masked product P_X V is skipped for key tiles where no row
+// of the CTA has an allowed key. Each CTA reduces sum((O_X - O_full)^2) over
+// its rows in a fixed order into the workspace; a second kernel adds the
+// tiles in a fixed order and labels the head.
 #include "internal.h"
 #include "sm100.cuh"
 
 namespace svg {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;
 constexpr int kTile = 128;  // sampled rows per CTA and keys per tile
+constexpr int kHalf = 64;   // keys per softmax thread per tile
 constexpr float kRebaseLog2 = 8.0f;
+
+struct PBarriers {
+  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full, o_final, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int x_active[2][kSoftmaxWarps];
+  float xmax[2][2][128];  // [half][full, masked][row]
+  float xsum[2][2][128];  // [half][full, masked][row]
+  float red[2][128];
+  int pair_fail[4][2];
+};
 
 template <int D>
 struct PCfg {
@@ -38,11 +62,13 @@ struct PCfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
   static constexpr int kOffBar = kOffV + kStages * kKVBytes;
-  static constexpr int kBarBytes = 1024;
+  static constexpr int kBarBytes = (static_cast<int>(sizeof(PBarriers)) + 127) / 128 * 128;
   static constexpr int kUsed = kOffBar + kBarBytes + 1024;
   static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColOF = 256, kColOX = 256 + D;
+  static_assert(kOffBar + kBarBytes + 1024 <= kSmem, "bookkeeping must fit the allocation");
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
 
 struct __align__(64) ProfParams {
@@ -56,20 +82,16 @@ struct __align__(64) ProfParams {
   float scale_log2;
 };
 
-struct PBarriers {
-  uint64_t k_full[3], v_full[3], kv_empty[3];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_full, o_final, drain;
-  uint32_t tmem_base;
-  int abort_flag;
-  int x_active[2][4];
-  float red[128];
-};
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
-__device__ __forceinline__ void named_sync_softmax() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+// Barrier of the two warps that share a group of 32 rows (ids 1..4).
+__device__ __forceinline__ void pair_sync(int group) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + group) : "memory");
+}
+
+__device__ __forceinline__ void softmax_sync() {
+  asm volatile("bar.sync 5, 256;" ::: "memory");
 }
 
 template <int D>
@@ -104,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->p_full[s], 128);
+      mbar_init(&bar->p_full[s], 32 * kSoftmaxWarps);
     }
     mbar_init(&bar->o_full, 1);
     mbar_init(&bar->o_final, 1);
@@ -112,26 +134,30 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     bar->abort_flag = 0;
     fence_mbar_init();
   }
-  // Gather the sampled Q rows into the swizzled K-major tile (rows past the
-  // sample count, and out-of-range indices, become zero rows).
+  // Gather the sampled Q rows into the swizzled K-major tile: row r = tid % 128,
+  // half h = tid / 128 copies 16-byte chunks [h*D/16, (h+1)*D/16). Rows past the
+  // sample count, and out-of-range indices, become zero rows.
+  const int row = tid & 127;
+  const int half = (tid >> 7) & 1;
   int qrow = -1;
-  if (tid < 128) {
-    const int si = tile * kTile + tid;
+  if (warp < kSoftmaxWarps) {
+    const int si = tile * kTile + row;
     if (si < p.n_samples) {
       const int r = __ldg(p.sample_idx + si);
       if (r >= 0 && r < p.Nv) {
         qrow = r;
-      } else {
+      } else if (half == 0) {
         atomicOr(p.status, kDevErrBounds);
       }
     }
     const uint4* src = reinterpret_cast<const uint4*>(
         p.q + (static_cast<size_t>(bh) * p.N + (qrow >= 0 ? qrow : 0)) * D);
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
+    for (int cc = 0; cc < D / 16; ++cc) {
+      const int c = half * (D / 16) + cc;
       const uint4 v = qrow >= 0 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-      const int pn = c >> 3, cc = c & 7;
-      *reinterpret_cast<uint4*>(sQ + pn * C::kPanel + tid * 128 + ((cc ^ (tid & 7)) << 4)) = v;
+      const int pn = c >> 3, ci = c & 7;
+      *reinterpret_cast<uint4*>(sQ + pn * C::kPanel + row * 128 + ((ci ^ (row & 7)) << 4)) = v;
     }
     fence_proxy_async_smem();
   }
@@ -200,7 +226,9 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
           if (!mbar_wait(&bar->v_full[st], (jj / C::kStages) & 1, abort_flag, p.status)) break;
           tc_fence_after();
           const volatile int* xa = bar->x_active[sb];
-          const bool x_on = (xa[0] | xa[1] | xa[2] | xa[3]) != 0;
+          int x_any = 0;
+#pragma unroll
+          for (int w = 0; w < kSoftmaxWarps; ++w) x_any |= xa[w];
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
             const uint64_t b = sdesc_sw128(v_addr + st * C::kKVBytes + kk * 16 * 128, C::kPanel,
@@ -208,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
             mma_bf16_ts(tmem + C::kColOF, p_col + kk * 8, b, idesc_pv,
                         (jj > 0 || kk > 0) ? 1u : 0u);
           }
-          if (x_on) {
+          if (x_any) {
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk) {
               const uint64_t b = sdesc_sw128(v_addr + st * C::kKVBytes + kk * 16 * 128,
@@ -232,67 +260,97 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int group = warp & 3;  // rows 32*group .. +31 (TMEM lane quarter)
+    const int c_base = half * kHalf;  // this thread's key columns within a tile
     const bool row_valid = qrow >= 0;
     const int qi = row_valid ? qrow : 0;
     const int f_i = qi / p.P;
     const int p_i = qi - f_i * p.P;
-    // spatial: allowed video keys are the frames [f_i - s, f_i + s], one index run
+    // Allowed video keys of this row: spatial = the frames [f_i - s, f_i + s]
+    // (one index run); temporal = positions [p_i - w, p_i + w] of every frame
+    // (one run per frame). Text keys [Nv, N) are allowed by both.
     const long long s_lo = static_cast<long long>(max(f_i - p.s, 0)) * p.P;
     const long long s_hi = static_cast<long long>(min(static_cast<long long>(f_i) + p.s + 1,
                                                       static_cast<long long>(p.T))) * p.P;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int t_lo = max(p_i - p.w, 0);
+    const int t_hi = static_cast<int>(
+        min(static_cast<long long>(p_i) + p.w, static_cast<long long>(p.P - 1)));
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(group * 32) << 16);
     float mF = -INFINITY, lF = 0.0f, mX = -INFINITY, lX = 0.0f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int sb = j & 1;
       const uint32_t s_col = lane_base + (sb ? C::kColS1 : C::kColS0);
-      const int j0 = j * kTile;
-      int kvalid = p.N - j0;
-      if (kvalid > kTile) kvalid = kTile;
-      // allowed-key bits of this row for the 128 keys of the tile
-      uint32_t bits[4] = {0u, 0u, 0u, 0u};
-      if (X == 0) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          const int jj = j0 + c;
-          const bool in = c < kvalid && (jj >= p.Nv || (jj >= s_lo && jj < s_hi));
-          bits[c >> 5] |= (in ? 1u : 0u) << (c & 31);
-        }
-      } else {
-        int pj = j0 % p.P;
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          const int jj = j0 + c;
-          const int dp = pj - p_i;
-          const bool in = c < kvalid && (jj >= p.Nv || (dp <= p.w && -dp <= p.w));
-          bits[c >> 5] |= (in ? 1u : 0u) << (c & 31);
-          pj = (pj + 1 == p.P) ? 0 : pj + 1;
+      const int k0 = j * kTile + c_base;       // first key of this thread's half
+      const int kvalid = max(0, min(kHalf, p.N - k0));
+      const int k_end = k0 + kvalid;           // exclusive
+      uint32_t bits[4] = {0u, 0u, 0u, 0u};     // only bits [0, 64) are used
+      if (row_valid && kvalid > 0) {
+        if (k_end > p.Nv) set_bit_range128(bits, max(p.Nv, k0) - k0, kvalid);
+        if (k0 < p.Nv) {
+          const int v_end = min(k_end, p.Nv);
+          if (X == 0) {
+            const long long a = max(s_lo, static_cast<long long>(k0));
+            const long long b = min(s_hi, static_cast<long long>(v_end));
+            if (b > a) set_bit_range128(bits, static_cast<int>(a - k0), static_cast<int>(b - k0));
+          } else {
+            for (int f = k0 / p.P; f * p.P < v_end; ++f) {
+              const long long a = static_cast<long long>(f) * p.P + t_lo;
+              const long long b = static_cast<long long>(f) * p.P + t_hi + 1;
+              const long long ca = max(a, static_cast<long long>(k0));
+              const long long cb = min(b, static_cast<long long>(v_end));
+              if (cb > ca)
+                set_bit_range128(bits, static_cast<int>(ca - k0), static_cast<int>(cb - k0));
+            }
+          }
         }
       }
-      if (!row_valid) bits[0] = bits[1] = bits[2] = bits[3] = 0u;
-      const bool any_x = (bits[0] | bits[1] | bits[2] | bits[3]) != 0u;
+      const bool any_x = (bits[0] | bits[1]) != 0u;
       const int warp_any = __any_sync(0xffffffffu, any_x) ? 1 : 0;
 
-      if (!mbar_wait(&bar->s_full[sb], (j >> 1) & 1, abort_flag, p.status)) {
+      if (ok && !mbar_wait(&bar->s_full[sb], (j >> 1) & 1, abort_flag, p.status)) ok = false;
+      // Both warps of a pair must take the same path through pair_sync (an
+      // unbounded barrier), so they agree on leaving the loop through it.
+      if (__any_sync(0xffffffffu, !ok)) ok = false;
+      if (lane_id() == 0) bar->pair_fail[group][half] = ok ? 0 : 1;
+      float a0 = -INFINITY, a1 = -INFINITY, b0 = -INFINITY, b1 = -INFINITY;
+      uint32_t sr[kHalf];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld_32x32b_x32(s_col + c_base, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld_32x32b_x32(s_col + c_base + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld_wait();
+        reg_fence(sr);
+        if (kvalid < kHalf) {  // only the last tile is ragged
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c)
+            if (c >= kvalid) sr[c] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int c = 0; c < kHalf; c += 4) {
+          a0 = fmax3(a0, u2f(sr[c]), u2f(sr[c + 1]));
+          a1 = fmax3(a1, u2f(sr[c + 2]), u2f(sr[c + 3]));
+          const float x0 = ((bits[c >> 5] >> (c & 31)) & 1u) ? u2f(sr[c]) : -INFINITY;
+          const float x1 = ((bits[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) ? u2f(sr[c + 1]) : -INFINITY;
+          const float x2 = ((bits[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u) ? u2f(sr[c + 2]) : -INFINITY;
+          const float x3 = ((bits[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u) ? u2f(sr[c + 3]) : -INFINITY;
+          b0 = fmax3(b0, x0, x1);
+          b1 = fmax3(b1, x2, x3);
+        }
+      }
+      // exchange the half-row maxima with the partner warp
+      bar->xmax[half][0][row] = fmaxf(a0, a1);
+      bar->xmax[half][1][row] = fmaxf(b0, b1);
+      pair_sync(group);
+      const float tF = fmaxf(bar->xmax[0][0][row], bar->xmax[1][0][row]) * p.scale_log2;
+      const float tX = fmaxf(bar->xmax[0][1][row], bar->xmax[1][1][row]) * p.scale_log2;
+      const int pair_failed = bar->pair_fail[group][0] | bar->pair_fail[group][1];
+      pair_sync(group);  // the exchange slots are rewritten next tile
+      if (pair_failed) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      uint32_t sr[kTile];
-#pragma unroll
-      for (int ch = 0; ch < kTile / 32; ++ch)
-        tmem_ld_32x32b_x32(s_col + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
-      tmem_ld_wait();
-      reg_fence(sr);
 
-      float mxF = -INFINITY, mxX = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const float x = u2f(sr[c]);
-        if (c < kvalid) mxF = fmaxf(mxF, x);
-        if ((bits[c >> 5] >> (c & 31)) & 1u) mxX = fmaxf(mxX, x);
-      }
-      const float tF = mxF * p.scale_log2, tX = mxX * p.scale_log2;
       const bool rbF = tF > mF + kRebaseLog2;
       const bool rbX = tX > mX + kRebaseLog2;
       const float mF_new = rbF ? tF : mF, mX_new = rbX ? tX : mX;
@@ -300,65 +358,68 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       const float aX = rbX ? fast_exp2(mX - mX_new) : 1.0f;
       const float uF = mF_new == -INFINITY ? 0.0f : mF_new;
       const float uX = mX_new == -INFINITY ? 0.0f : mX_new;
-      float sumF = 0.0f, sumX = 0.0f;
+      // P_X = P_full * 2^(mF - mX) on allowed keys, unless the masked base is
+      // so far below the full one that 2^(x - mF) could flush to zero; those
+      // (rare) warps evaluate the masked exponentials directly.
+      const float gap = uF - uX;
+      const bool direct = gap > 64.0f;
+      const float kX = direct ? 0.0f : fast_exp2(gap);
+      const bool warp_direct = __any_sync(0xffffffffu, direct);
+      float sF0 = 0.0f, sF1 = 0.0f, sX0 = 0.0f, sX1 = 0.0f;
 #pragma unroll
-      for (int ch = 0; ch < kTile / 32; ++ch) {
+      for (int ch = 0; ch < kHalf / 32; ++ch) {
         uint32_t pkF[16], pkX[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c0 = ch * 32 + 2 * i;
-          const float x0 = u2f(sr[c0]), x1 = u2f(sr[c0 + 1]);
-          const float f0 = c0 < kvalid ? fast_exp2(fmaf(x0, p.scale_log2, -uF)) : 0.0f;
-          const float f1 = c0 + 1 < kvalid ? fast_exp2(fmaf(x1, p.scale_log2, -uF)) : 0.0f;
+          float y0, y1;
+          ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
+          const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
           const bool in0 = (bits[ch] >> (2 * i)) & 1u;
           const bool in1 = (bits[ch] >> (2 * i + 1)) & 1u;
-          const float g0 = in0 ? fast_exp2(fmaf(x0, p.scale_log2, -uX)) : 0.0f;
-          const float g1 = in1 ? fast_exp2(fmaf(x1, p.scale_log2, -uX)) : 0.0f;
-          sumF += f0 + f1;
-          sumX += g0 + g1;
+          float g0 = in0 ? f0 * kX : 0.0f;
+          float g1 = in1 ? f1 * kX : 0.0f;
+          if (warp_direct && direct) {
+            g0 = in0 ? fast_exp2(fmaf(u2f(sr[c0]), p.scale_log2, -uX)) : 0.0f;
+            g1 = in1 ? fast_exp2(fmaf(u2f(sr[c0 + 1]), p.scale_log2, -uX)) : 0.0f;
+          }
+          fadd2(sF0, sF1, sF0, sF1, f0, f1);
+          fadd2(sX0, sX1, sX0, sX1, g0, g1);
           pkF[i] = pack_bf16x2(f0, f1);
           pkX[i] = pack_bf16x2(g0, g1);
         }
-        tmem_st_32x32b_x16(s_col + ch * 16, pkF);
-        tmem_st_32x32b_x16(s_col + 64 + ch * 16, pkX);
+        // keys k -> column k/2: this half's 64 keys fill 32 columns
+        tmem_st_32x32b_x16(s_col + half * 32 + ch * 16, pkF);
+        tmem_st_32x32b_x16(s_col + 64 + half * 32 + ch * 16, pkX);
       }
-      lF = lF * aF + sumF;
-      lX = lX * aX + sumX;
+      lF = lF * aF + (sF0 + sF1);
+      lX = lX * aX + (sX0 + sX1);
       mF = mF_new;
       mX = mX_new;
       tmem_st_wait();
       if (lane_id() == 0) bar->x_active[sb][warp] = warp_any;
 
+      // Re-base this half's columns of O_full / O_X once PV_{j-1} has landed.
       const bool wF = __any_sync(0xffffffffu, rbF);
       const bool wX = __any_sync(0xffffffffu, rbX);
       if (j > 0 && (wF || wX)) {
-        if (!mbar_wait(&bar->o_full, (j - 1) & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
+        // A failed wait is reported through the pair exchange of the next tile.
+        if (!mbar_wait(&bar->o_full, (j - 1) & 1, abort_flag, p.status)) ok = false;
         tc_fence_after();
-        if (wF) {
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
+        for (int which = 0; which < 2 && ok; ++which) {
+          if (which == 0 ? !wF : !wX) continue;
+          const float a = which == 0 ? aF : aX;
+          const uint32_t ocol = lane_base + (which == 0 ? C::kColOF : C::kColOX) + half * (D / 2);
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
             uint32_t o[32];
-            tmem_ld_32x32b_x32(lane_base + C::kColOF + ch * 32, o);
+            tmem_ld_32x32b_x32(ocol + ch * 32, o);
             tmem_ld_wait();
             reg_fence(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * aF);
-            tmem_st_32x32b_x32(lane_base + C::kColOF + ch * 32, o);
-          }
-        }
-        if (wX) {
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld_32x32b_x32(lane_base + C::kColOX + ch * 32, o);
-            tmem_ld_wait();
-            reg_fence(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * aX);
-            tmem_st_32x32b_x32(lane_base + C::kColOX + ch * 32, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * a);
+            tmem_st_32x32b_x32(ocol + ch * 32, o);
           }
         }
         tmem_st_wait();
@@ -367,18 +428,24 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       mbar_arrive(&bar->p_full[sb]);
     }
 
-    // ---- per-row squared error, then a fixed-order CTA sum
+    // ---- per-row squared error over this half's d/2 channels
+    bar->xsum[half][0][row] = lF;
+    bar->xsum[half][1][row] = lX;
     if (ok && n > 0) ok = mbar_wait(&bar->o_final, 0, abort_flag, p.status);
+    softmax_sync();
+    const float LF = bar->xsum[0][0][row] + bar->xsum[1][0][row];
+    const float LX = bar->xsum[0][1][row] + bar->xsum[1][1][row];
     tc_fence_after();
     float err = 0.0f;
-    if (ok && n > 0) {
-      const float iF = lF > 0.0f ? 1.0f / lF : 0.0f;
-      const float iX = lX > 0.0f ? 1.0f / lX : 0.0f;
+    const bool all_ok = __all_sync(0xffffffffu, ok);
+    if (all_ok && n > 0) {
+      const float iF = LF > 0.0f ? 1.0f / LF : 0.0f;
+      const float iX = LX > 0.0f ? 1.0f / LX : 0.0f;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = 0; ch < D / 64; ++ch) {
         uint32_t oF[32], oX[32];
-        tmem_ld_32x32b_x32(lane_base + C::kColOF + ch * 32, oF);
-        tmem_ld_32x32b_x32(lane_base + C::kColOX + ch * 32, oX);
+        tmem_ld_32x32b_x32(lane_base + C::kColOF + half * (D / 2) + ch * 32, oF);
+        tmem_ld_32x32b_x32(lane_base + C::kColOX + half * (D / 2) + ch * 32, oX);
         tmem_ld_wait();
         reg_fence(oF);
         reg_fence(oX);
@@ -389,12 +456,14 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
         }
       }
     }
-    bar->red[tid] = row_valid ? err : 0.0f;
-    named_sync_softmax();
+    bar->red[half][row] = row_valid ? err : 0.0f;
+    if (!all_ok) atomicOr(&bar->abort_flag, 1);
+    softmax_sync();
     if (tid == 0) {
       float acc = 0.0f;
-      for (int i = 0; i < 128; ++i) acc += bar->red[i];
-      p.partial[(static_cast<size_t>(bh) * 2 + X) * p.n_tiles + tile] = ok ? acc : __int_as_float(0x7fc00000);
+      for (int i = 0; i < 128; ++i) acc += bar->red[0][i] + bar->red[1][i];
+      p.partial[(static_cast<size_t>(bh) * 2 + X) * p.n_tiles + tile] =
+          *abort_flag ? __int_as_float(0x7fc00000) : acc;
     }
   }
 

@@ -267,6 +267,48 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input form).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pairs: one instruction computes both lanes.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                      float c0, float c1) {
+  uint64_t a, b, c, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(c0), "f"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  uint64_t a, b, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
+// Sets bits [a, b) (clipped to [0, 128)) of a 128-bit set held in 4 words.
+__device__ __forceinline__ void set_bit_range128(uint32_t (&w)[4], int a, int b) {
+  a = a < 0 ? 0 : a;
+  b = b > 128 ? 128 : b;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int lo = a - 32 * i < 0 ? 0 : a - 32 * i;
+    const int hi = b - 32 * i > 32 ? 32 : b - 32 * i;
+    if (hi > lo) {
+      const uint32_t span = hi - lo == 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u);
+      w[i] |= span << lo;
+    }
+  }
+}
+
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 __device__ __forceinline__ bool elect_one() {
