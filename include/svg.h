@@ -137,6 +137,37 @@ svg_status svg_profile_heads(const svg_geom* geom, const svg_bf16* q, const svg_
                              size_t workspace_bytes, svg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * svg_profile_heads_noalloc -- svg_profile_heads without a caller workspace.
+ * No counterpart on the pages: this is an interface convenience, not part of
+ * the method. Some callers cannot allocate device memory when they call the
+ * library: a plugin inside an inference engine that plans every buffer up
+ * front and forbids allocation in its execute path, a latency-critical loop
+ * that cannot afford cudaMalloc's implicit device synchronisation, or code
+ * that simply has no allocator at hand. This entry point takes the same
+ * arguments as svg_profile_heads minus the workspace and keeps the MSE
+ * partial sums in a fixed array inside the library instead; it calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   Limit      the partial sums need B*H*2*ceil(n_samples/128)*4 bytes
+ *              (svg_profile_workspace_bytes); more than 256 KiB (that is,
+ *              B*H*ceil(n_samples/128) > 32768) returns SVG_ERR_CAPACITY
+ *              before anything is launched.
+ *   Memory     every GPU that loads the library holds the 256 KiB array
+ *              until the process exits.
+ *   Set-up     the first call on a device looks up that device's copy of
+ *              the array (cudaGetSymbolAddress) with the device current;
+ *              make that first call before any stream capture.
+ *   Sharing    all calls share the one array and it keeps the last call's
+ *              contents (every slot is written before it is read, so no
+ *              clearing is needed); calls that overlap on the GPU (e.g. on
+ *              two streams) race and must be serialised by the caller.
+ * Errors: as svg_profile_heads (CAPACITY as above).
+ */
+svg_status svg_profile_heads_noalloc(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                                     const svg_bf16* v, const int32_t* sample_idx,
+                                     int32_t n_samples, int8_t* labels, float* mse,
+                                     svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * svg_permute / svg_unpermute -- the layout transformation (SVG abstract:
  * "hardware-efficient tensor layout transformation").
  *   permute:    out[b,h,pi(i),:] = in[b,h,i,:]   (frame-major -> position-major)

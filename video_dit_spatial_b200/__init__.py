@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "SVG_OK", 1: "SVG_ERR_INVALID_ARG", 2: "SVG_ERR_UNSUPPORTED",
 
 EXPORTED = [
     "svg_mask_nnz", "svg_build_block_mask", "svg_profile_workspace_bytes",
-    "svg_profile_heads", "svg_permute", "svg_unpermute", "svg_permute_qkv",
+    "svg_profile_heads", "svg_profile_heads_noalloc", "svg_permute", "svg_unpermute", "svg_permute_qkv",
     "svg_sparse_attention", "svg_get_device_status", "svg_selftest_wait_timeout",
     "svg_status_string", "svg_version",
 ]
@@ -95,6 +95,7 @@ def load() -> ctypes.CDLL:
         "svg_build_block_mask": [_c_geom_p, _i32, _vp, _vp, _i64, _vp],
         "svg_profile_workspace_bytes": [_c_geom_p, _i32, ctypes.POINTER(_sz)],
         "svg_profile_heads": [_c_geom_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp],
+        "svg_profile_heads_noalloc": [_c_geom_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp],
         "svg_permute": [_c_geom_p, _vp, _vp, _vp, _vp],
         "svg_unpermute": [_c_geom_p, _vp, _vp, _vp, _vp],
         "svg_permute_qkv": [_c_geom_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
@@ -171,6 +172,15 @@ def svg_profile_heads(geom: Geom, q, k, v, sample_idx, labels, mse=None, workspa
     _check("svg_profile_heads", load().svg_profile_heads(
         ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(sample_idx), n, _ptr(labels),
         _ptr(mse), _ptr(workspace), wb, _stream(stream)))
+
+
+def svg_profile_heads_noalloc(geom: Geom, q, k, v, sample_idx, labels, mse=None,
+                              n_samples=None, stream=None) -> None:
+    """svg_profile_heads with the library's fixed internal scratch (no workspace)."""
+    n = sample_idx.numel() if n_samples is None else n_samples
+    _check("svg_profile_heads_noalloc", load().svg_profile_heads_noalloc(
+        ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(sample_idx), n, _ptr(labels),
+        _ptr(mse), _stream(stream)))
 
 
 def svg_permute(geom: Geom, inp, out, labels=None, stream=None) -> None:

@@ -227,6 +227,30 @@ svg_status svg_profile_heads(const svg_geom* geom, const svg_bf16* q, const svg_
   return SVG_OK;
 }
 
+svg_status svg_profile_heads_noalloc(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                                     const svg_bf16* v, const int32_t* sample_idx,
+                                     int32_t n_samples, int8_t* labels, float* mse,
+                                     svg_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || sample_idx == nullptr || labels == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  if (!svg::aligned16(q) || !svg::aligned16(k) || !svg::aligned16(v)) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_geom(geom, true);
+  if (st != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  if (n_samples < 1 || n_samples > d.Nv) return SVG_ERR_INVALID_ARG;
+  size_t need = 0;
+  svg_profile_workspace_bytes(geom, n_samples, &need);
+  if (need > svg::profile_noalloc_scratch_bytes()) return SVG_ERR_CAPACITY;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  svg::ProfileArgs a{q, k, v, sample_idx, n_samples, labels, mse, nullptr};
+  if (svg::launch_profile_noalloc(d, a, status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SVG_ERR_CUDA;
+  return SVG_OK;
+}
+
 static svg_status permute_common(const svg_geom* geom, int n, const svg_bf16* const* in,
                                  svg_bf16* const* out, const int8_t* labels, bool inverse,
                                  svg_stream_t stream) {

@@ -114,6 +114,11 @@ struct ProfileArgs {
 };
 int32_t profile_tiles(int32_t n_samples);
 cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cudaStream_t stream);
+// Same launch with the partial sums in the module's fixed device scratch
+// (a.partial is ignored); see svg_profile_heads_noalloc.
+size_t profile_noalloc_scratch_bytes();
+cudaError_t launch_profile_noalloc(const Dims& d, const ProfileArgs& a, int* status,
+                                   cudaStream_t stream);
 
 cudaError_t launch_wait_selftest(long long limit_cycles, int* status, cudaStream_t stream);
 

@@ -24,6 +24,8 @@
 // of the CTA has an allowed key. Each CTA reduces sum((O_X - O_full)^2) over
 // its rows in a fixed order into the workspace; a second kernel adds the
 // tiles in a fixed order and labels the head.
+#include <mutex>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -514,6 +516,52 @@ cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, flo
 }  // namespace
 
 int32_t profile_tiles(int32_t n_samples) { return (n_samples + kTile - 1) / kTile; }
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for svg_profile_heads_noalloc: the per-tile partial sums live
+// in this module's own device array instead of caller memory. Every GPU that
+// loads the library keeps one copy until the process exits. The profiling
+// kernel writes every slot it later reads, so nothing needs clearing between
+// calls; calls that overlap on the GPU share it and race.
+namespace {
+constexpr size_t kNoAllocScratchBytes = 256 * 1024;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+float* g_scratch_ptr[kMaxScratchDevices] = {};
+
+// Device address of the current device's copy of g_noalloc_scratch. In host
+// code the array's name is only a stand-in, so the address is looked up with
+// cudaGetSymbolAddress, once per device, with that device current.
+cudaError_t noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+size_t profile_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_profile_noalloc(const Dims& d, const ProfileArgs& a, int* status,
+                                   cudaStream_t stream) {
+  float* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  ProfileArgs args = a;
+  args.partial = scratch;
+  return launch_profile(d, args, status, stream);
+}
 
 cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cudaStream_t stream) {
   ProfParams pp;
