@@ -50,6 +50,25 @@ def _peaks():
             "source": "fallback"}
 
 
+def _captured_traffic():
+    """DRAM bytes per full-size attention launch from the committed ncu summary,
+    or None when the kernel sources changed since that capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "sparse_attention_pair_hunyuan_H4_d128.md")
+    srcs = [os.path.join(ROOT, "video_dit_spatial_b200", "csrc", f)
+            for f in ("attention.cu", "sm100.cuh")]
+    try:
+        text = open(path).read()
+        digest = hashlib.sha256(b"".join(open(f, "rb").read() for f in srcs)).hexdigest()[:16]
+    except OSError:
+        return None
+    fields = dict(line.strip().split(": ", 1) for line in text.splitlines()
+                  if line.strip().startswith(("traffic_bytes", "kernel_sources")))
+    if fields.get("kernel_sources_sha256_16") != digest:
+        return None
+    return int(fields["traffic_bytes_per_launch_full_size"])
+
+
 def _dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -204,6 +223,46 @@ def run_reference(args, wl):
 
 
 # ---------------------------------------------------------------------------
+# small-case driver for ncu captures
+# ---------------------------------------------------------------------------
+def run_capture(args, wl):
+    """One kernel, three launches, on the workload cut to --heads heads (the
+    planted head split kept at half spatial); inputs stay larger than L2."""
+    import video_dit_spatial_b200 as svg
+    from video_dit_spatial_b200.layer import SparseVideoGenLayer
+    wl = wl.replace(H=args.heads, n_spatial=args.heads // 2)
+    g = svg.Geom.from_workload(wl)
+    q, k, v = (t.cuda() for t in SI.make_qkv(wl))
+    rows = SI.sample_rows(wl).cuda()
+    layer = SparseVideoGenLayer(g, wl.n_samples)
+    o = torch.empty_like(q)
+    layer.build_masks()
+    layer.labels.copy_(torch.tensor(SI.planted_head_kinds(wl) * wl.B, dtype=torch.int8))
+    if args.capture == "attention":
+        svg.svg_permute_qkv(g, q, k, v, layer.qp, layer.kp, layer.vp, layer.labels)
+    fns = {
+        "attention": lambda: svg.svg_sparse_attention(
+            g, q, k, v, layer.qp, layer.kp, layer.vp, layer.labels,
+            layer.masks[0].row_ptr, layer.masks[0].col_idx, layer.masks[1].row_ptr,
+            layer.masks[1].col_idx, o, layer.op),
+        "profile": lambda: layer.profile(q, k, v, rows),
+        "permute": lambda: svg.svg_permute_qkv(g, q, k, v, layer.qp, layer.kp, layer.vp,
+                                               layer.labels),
+    }
+    fn = fns[args.capture]
+    for it in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        print(f"{args.capture} {wl.name} H={wl.H} launch {it}: {e0.elapsed_time(e1):.3f} ms")
+    st, bits = svg.svg_get_device_status()
+    if st != svg.SVG_OK:
+        raise RuntimeError(f"device status {st} bits {bits}")
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def main():
@@ -216,10 +275,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--capture", choices=["attention", "profile", "permute"],
+                    help="small case for an ncu capture: run one kernel 3 times on the "
+                         "workload with --heads heads, print per-launch ms, no JSON line")
+    ap.add_argument("--heads", type=int, default=4)
     args = ap.parse_args()
     wl = SI.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)
+        return
+    if args.capture:
+        run_capture(args, wl)
         return
     if args.warmup < 3:
         args.warmup = 3
@@ -352,7 +418,8 @@ def main():
                 "frac": achieved / pk["bf16_tflops_sustained"],
                 "peak_kind": f"bf16 dense, sustained, {pk['source']}",
                 "frac_of_burst_peak": achieved / pk["bf16_tflops"],
-                "traffic": None}
+                "traffic": _captured_traffic() if wl.name == SI.HUNYUAN.name else None,
+                "traffic_note": "ncu dram read+write of a 4-head launch, scaled by heads"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
