@@ -69,7 +69,7 @@ struct __align__(64) AttnParams {
   svg_bf16* out[2];
   float* lse;
   int* status;
-  int32_t N, BH, nqb, nkb, bq, bk;
+  int32_t N, Nv, BH, nqb, nkb, bq, bk;
   int32_t has_permuted;
   float scale_log2;
 };
@@ -383,6 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kPairThreads = 384;
 constexpr int kPairProducerWarp = 8;
 constexpr int kPairMmaWarp = 9;
+// One exp2 pair in kPairEmuEvery on the FMA pipe (0 = all on MUFU). Measured
+// on the HunyuanVideo-shaped layer: 1 in 4 made the kernel slower (28.2 ->
+// 33.5 ms): the softmax is bound by its per-tile critical path, not by MUFU.
+constexpr int kPairEmuEvery = 0;
 constexpr int kPairLaunchRegs = 168;   // per thread at launch (3 warps per sub-partition)
 constexpr int kPairSoftmaxRegs = 224;  // softmax warpgroups after setmaxnreg.inc
 constexpr int kPairOtherRegs = 56;     // producer / MMA warpgroup after setmaxnreg.dec
@@ -454,9 +458,24 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  // Work order (1-D grid): first the pairs holding text rows (dense rows, by far
+  // the longest) of every head, so none of them starts near the end; then the
+  // remaining pairs head by head, last pair first, so the CTAs running at the
+  // same time share one head's K/V window in L2.
   const int npairs = (p.nqb + 1) >> 1;
-  const int pair = npairs - 1 - static_cast<int>(blockIdx.x);  // text-heavy rows first
-  const int bh = blockIdx.y;
+  const int first_text_pair = (p.Nv / 128) >> 1;  // pair holding the first text row
+  const int n_long = npairs - first_text_pair;
+  const int lin = static_cast<int>(blockIdx.x);
+  int pair, bh;
+  if (lin < n_long * p.BH) {
+    bh = lin % p.BH;
+    pair = npairs - 1 - lin / p.BH;
+  } else {
+    const int rest = lin - n_long * p.BH;
+    const int per_head = npairs - n_long;
+    bh = rest / per_head;
+    pair = per_head - 1 - rest % per_head;
+  }
 
   const int label = p.labels ? static_cast<int>(p.labels[bh]) : SVG_HEAD_SPATIAL;
   const int sel = label == SVG_HEAD_TEMPORAL ? 1 : 0;
@@ -678,29 +697,42 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int i = 0; i < BK; ++i)
           if (i >= kvalid) sr[i] = __float_as_uint(-INFINITY);
       }
-      float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+      // row maximum: eight independent 3-input max chains, then a small tree
+      float xm[8];
 #pragma unroll
-      for (int i = 0; i < BK; i += 8) {
-        x0 = fmax3(x0, u2f(sr[i]), u2f(sr[i + 1]));
-        x1 = fmax3(x1, u2f(sr[i + 2]), u2f(sr[i + 3]));
-        x2 = fmax3(x2, u2f(sr[i + 4]), u2f(sr[i + 5]));
-        x3 = fmax3(x3, u2f(sr[i + 6]), u2f(sr[i + 7]));
+      for (int c = 0; c < 8; ++c) xm[c] = fmax3(u2f(sr[2 * c]), u2f(sr[2 * c + 1]), -INFINITY);
+#pragma unroll
+      for (int i = 16; i < BK; i += 16) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xm[c] = fmax3(xm[c], u2f(sr[i + 2 * c]), u2f(sr[i + 2 * c + 1]));
       }
-      const float m_tile = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)) * p.scale_log2;
+      const float m_tile =
+          fmaxf(fmax3(xm[0], xm[1], xm[2]), fmax3(xm[3], fmax3(xm[4], xm[5], xm[6]), xm[7])) *
+          p.scale_log2;
       const bool rebase = m_tile > m + kRebaseLog2;
       const float m_new = rebase ? m_tile : m;
       const float alpha = rebase ? fast_exp2(m - m_new) : 1.0f;  // exp2(-inf) = 0
       const float m_use = m_new == -INFINITY ? 0.0f : m_new;
       float s0 = 0.0f, s1 = 0.0f;
+      // Full tiles may evaluate one pair in kPairEmuEvery on the FMA pipe; the
+      // ragged tile uses MUFU only.
+      const bool full_tile = kvalid == BK;
 #pragma unroll
       for (int ch = 0; ch < BK / 32; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c0 = ch * 32 + 2 * i;
-          float y0, y1;
+          float y0, y1, e0, e1;
           ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -m_use, -m_use);
-          const float e0 = fast_exp2(y0), e1 = fast_exp2(y1);
+          bool emulate = false;
+          if constexpr (kPairEmuEvery > 0) emulate = full_tile && i % kPairEmuEvery == kPairEmuEvery - 1;
+          if (emulate) {
+            exp2_poly2(e0, e1, y0, y1);
+          } else {
+            e0 = fast_exp2(y0);
+            e1 = fast_exp2(y1);
+          }
           fadd2(s0, s1, s0, s1, e0, e1);
           pk[i] = pack_bf16x2(e0, e1);
         }
@@ -785,7 +817,7 @@ cudaError_t launch_pair(const Dims& d, const AttnParams& p, cudaStream_t stream)
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kPairThreads, C::kSmem);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kPairLaunchRegs || resident < 1) return launch_impl<D, BK>(d, p, stream);
-  dim3 grid((d.nqb + 1) / 2, d.BH);
+  dim3 grid(static_cast<unsigned>(((d.nqb + 1) / 2) * d.BH));
   kern<<<grid, kPairThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError();
 }
@@ -832,6 +864,7 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
   p.lse = a.lse;
   p.status = status;
   p.N = d.N;
+  p.Nv = d.Nv;
   p.BH = d.BH;
   p.nqb = d.nqb;
   p.nkb = d.nkb;
