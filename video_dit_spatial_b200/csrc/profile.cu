@@ -41,7 +41,7 @@ constexpr int kHalf = 64;   // keys per softmax thread per tile
 constexpr float kRebaseLog2 = 8.0f;
 
 struct PBarriers {
-  uint64_t k_full[3], v_full[3], kv_empty[3];
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
   uint64_t s_full[2], p_full[2];
   uint64_t o_full, o_final, drain;
   uint32_t tmem_base;
@@ -59,11 +59,14 @@ struct PCfg {
   static constexpr int kPanel = 128 * 128;  // 128 rows x 128 B
   static constexpr int kQBytes = kPanels * kPanel;
   static constexpr int kKVBytes = kPanels * kPanel;
-  static constexpr int kStages = D == 128 ? 2 : 3;
+  // K is released right after its QK product, V only after its PV products,
+  // so K gets the deeper ring.
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = D == 128 ? 2 : 3;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kKVBytes;
   static constexpr int kBarBytes = (static_cast<int>(sizeof(PBarriers)) + 127) / 128 * 128;
   static constexpr int kUsed = kOffBar + kBarBytes + 1024;
   static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
@@ -121,10 +124,11 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     tc_fence_before();
   }
   if (tid == 32) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_empty[s], 1);
       mbar_init(&bar->v_full[s], 1);
-      mbar_init(&bar->kv_empty[s], 1);
+      mbar_init(&bar->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->s_full[s], 1);
@@ -170,27 +174,44 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
   if (warp == kProducerWarp) {
     if (lane_id() == 0) {
       const uint64_t keep = l2_policy_evict_last();
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int st = j % C::kStages;
-        if (!mbar_wait(&bar->kv_empty[st], ((j / C::kStages) & 1) ^ 1, abort_flag, p.status))
-          break;
-        mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kPanel, &p.tm_k, &bar->k_full[st],
-                           pn * 64, j * kTile, bh, keep);
-        mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kPanel, &p.tm_v, &bar->v_full[st],
-                           pn * 64, j * kTile, bh, keep);
-        issued = j + 1;
+      // K runs up to kKStages tiles ahead, V up to kVStages; K(j) is issued
+      // before V(j-1) so the deeper K ring is used.
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % C::kKStages;
+          ok = mbar_wait(&bar->k_empty[st], ((j / C::kKStages) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kPanel, &p.tm_k, &bar->k_full[st],
+                             pn * 64, j * kTile, bh, keep);
+          k_issued = j + 1;
+        }
+        if (j >= 1) {
+          const int jv = j - 1;
+          const int st = jv % C::kVStages;
+          ok = mbar_wait(&bar->v_empty[st], ((jv / C::kVStages) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kPanel, &p.tm_v, &bar->v_full[st],
+                             pn * 64, jv * kTile, bh, keep);
+          v_issued = jv + 1;
+        }
       }
       if (*abort_flag) {
-        for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
-          const int st = j % C::kStages;
-          const uint32_t par = (j / C::kStages) & 1;
+        // Let every copy this thread started land before the CTA retires.
+        for (int j = (k_issued > C::kKStages ? k_issued - C::kKStages : 0); j < k_issued; ++j) {
           long long t0 = clock64();
-          while (!(mbar_try_wait(&bar->k_full[st], par) && mbar_try_wait(&bar->v_full[st], par)) &&
+          while (!mbar_try_wait(&bar->k_full[j % C::kKStages], (j / C::kKStages) & 1) &&
+                 clock64() - t0 < kWaitLimitCycles) {
+          }
+        }
+        for (int j = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); j < v_issued; ++j) {
+          long long t0 = clock64();
+          while (!mbar_try_wait(&bar->v_full[j % C::kVStages], (j / C::kVStages) & 1) &&
                  clock64() - t0 < kWaitLimitCycles) {
           }
         }
@@ -206,9 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       bool x_started = false;
       for (int j = 0; j <= n; ++j) {
         if (j < n) {
-          const int st = j % C::kStages;
+          const int st = j % C::kKStages;
           const uint32_t s_col = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
-          if (!mbar_wait(&bar->k_full[st], (j / C::kStages) & 1, abort_flag, p.status)) break;
+          if (!mbar_wait(&bar->k_full[st], (j / C::kKStages) & 1, abort_flag, p.status)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -218,14 +239,15 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
                         kk > 0 ? 1u : 0u);
           }
           tc_commit(&bar->s_full[j & 1]);
+          tc_commit(&bar->k_empty[st]);  // K(j) is free once QK_j retires
         }
         if (j >= 1) {
           const int jj = j - 1;
-          const int st = jj % C::kStages;
+          const int st = jj % C::kVStages;
           const int sb = jj & 1;
           const uint32_t p_col = tmem + (sb ? C::kColS1 : C::kColS0);
           if (!mbar_wait(&bar->p_full[sb], (jj >> 1) & 1, abort_flag, p.status)) break;
-          if (!mbar_wait(&bar->v_full[st], (jj / C::kStages) & 1, abort_flag, p.status)) break;
+          if (!mbar_wait(&bar->v_full[st], (jj / C::kVStages) & 1, abort_flag, p.status)) break;
           tc_fence_after();
           const volatile int* xa = bar->x_active[sb];
           int x_any = 0;
@@ -248,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
             }
             x_started = true;
           }
-          tc_commit(&bar->kv_empty[st]);
+          tc_commit(&bar->v_empty[st]);
           tc_commit(&bar->o_full);
           if (jj == n - 1) tc_commit(&bar->o_final);
         }
@@ -271,39 +293,35 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     // Allowed video keys of this row: spatial = the frames [f_i - s, f_i + s]
     // (one index run); temporal = positions [p_i - w, p_i + w] of every frame
     // (one run per frame). Text keys [Nv, N) are allowed by both.
-    const long long s_lo = static_cast<long long>(max(f_i - p.s, 0)) * p.P;
-    const long long s_hi = static_cast<long long>(min(static_cast<long long>(f_i) + p.s + 1,
-                                                      static_cast<long long>(p.T))) * p.P;
+    const int s_lo = max(f_i - p.s, 0) * p.P;  // frames [f_i - s, f_i + s] as one index run
+    const int s_hi = static_cast<int>(min(static_cast<long long>(f_i) + p.s + 1,
+                                          static_cast<long long>(p.T))) * p.P;
     const int t_lo = max(p_i - p.w, 0);
     const int t_hi = static_cast<int>(
         min(static_cast<long long>(p_i) + p.w, static_cast<long long>(p.P - 1)));
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(group * 32) << 16);
     float mF = -INFINITY, lF = 0.0f, mX = -INFINITY, lX = 0.0f;
     bool ok = true;
+    int fs0 = 0;  // start of the frame holding this thread's first key of the tile
     for (int j = 0; j < n; ++j) {
       const int sb = j & 1;
       const uint32_t s_col = lane_base + (sb ? C::kColS1 : C::kColS0);
       const int k0 = j * kTile + c_base;       // first key of this thread's half
       const int kvalid = max(0, min(kHalf, p.N - k0));
       const int k_end = k0 + kvalid;           // exclusive
-      uint32_t bits[4] = {0u, 0u, 0u, 0u};     // only bits [0, 64) are used
+      uint32_t bits[2] = {0u, 0u};  // allowed keys k0 + [0, 64) of this row
       if (row_valid && kvalid > 0) {
-        if (k_end > p.Nv) set_bit_range128(bits, max(p.Nv, k0) - k0, kvalid);
+        if (k_end > p.Nv) set_bit_range64(bits, max(p.Nv, k0) - k0, kvalid);
         if (k0 < p.Nv) {
           const int v_end = min(k_end, p.Nv);
           if (X == 0) {
-            const long long a = max(s_lo, static_cast<long long>(k0));
-            const long long b = min(s_hi, static_cast<long long>(v_end));
-            if (b > a) set_bit_range128(bits, static_cast<int>(a - k0), static_cast<int>(b - k0));
+            set_bit_range64(bits, max(s_lo, k0) - k0, min(s_hi, v_end) - k0);
           } else {
-            for (int f = k0 / p.P; f * p.P < v_end; ++f) {
-              const long long a = static_cast<long long>(f) * p.P + t_lo;
-              const long long b = static_cast<long long>(f) * p.P + t_hi + 1;
-              const long long ca = max(a, static_cast<long long>(k0));
-              const long long cb = min(b, static_cast<long long>(v_end));
-              if (cb > ca)
-                set_bit_range128(bits, static_cast<int>(ca - k0), static_cast<int>(cb - k0));
-            }
+            // frames overlapping the half tile (at most two when P >= 64);
+            // fs0 tracks the start of the frame holding k0 across tiles
+            while (fs0 + p.P <= k0) fs0 += p.P;
+            for (int fs = fs0; fs < v_end; fs += p.P)
+              set_bit_range64(bits, max(fs + t_lo, k0) - k0, min(fs + t_hi + 1, v_end) - k0);
           }
         }
       }
@@ -332,12 +350,21 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
         for (int c = 0; c < kHalf; c += 4) {
           a0 = fmax3(a0, u2f(sr[c]), u2f(sr[c + 1]));
           a1 = fmax3(a1, u2f(sr[c + 2]), u2f(sr[c + 3]));
-          const float x0 = ((bits[c >> 5] >> (c & 31)) & 1u) ? u2f(sr[c]) : -INFINITY;
-          const float x1 = ((bits[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) ? u2f(sr[c + 1]) : -INFINITY;
-          const float x2 = ((bits[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u) ? u2f(sr[c + 2]) : -INFINITY;
-          const float x3 = ((bits[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u) ? u2f(sr[c + 3]) : -INFINITY;
-          b0 = fmax3(b0, x0, x1);
-          b1 = fmax3(b1, x2, x3);
+        }
+        // The masked maximum of this half can only move the masked base when
+        // the half's full maximum exceeds mX + 2^8; otherwise report -inf: the
+        // combined decision and the new base are unchanged.
+        const bool need_m = any_x && fmaxf(a0, a1) * p.scale_log2 > mX + kRebaseLog2;
+        if (__any_sync(0xffffffffu, need_m)) {
+#pragma unroll
+          for (int c = 0; c < kHalf; c += 4) {
+            const float x0 = ((bits[c >> 5] >> (c & 31)) & 1u) ? u2f(sr[c]) : -INFINITY;
+            const float x1 = ((bits[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) ? u2f(sr[c + 1]) : -INFINITY;
+            const float x2 = ((bits[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u) ? u2f(sr[c + 2]) : -INFINITY;
+            const float x3 = ((bits[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u) ? u2f(sr[c + 3]) : -INFINITY;
+            b0 = fmax3(b0, x0, x1);
+            b1 = fmax3(b1, x2, x3);
+          }
         }
       }
       // exchange the half-row maxima with the partner warp
@@ -363,32 +390,77 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       // P_X = P_full * 2^(mF - mX) on allowed keys, unless the masked base is
       // so far below the full one that 2^(x - mF) could flush to zero; those
       // (rare) warps evaluate the masked exponentials directly.
+      // (With no allowed key seen yet, mX is -inf and every P_X is zero.)
       const float gap = uF - uX;
-      const bool direct = gap > 64.0f;
+      const bool direct = mX_new != -INFINITY && gap > 64.0f;
       const float kX = direct ? 0.0f : fast_exp2(gap);
       const bool warp_direct = __any_sync(0xffffffffu, direct);
+      // Warp-uniform shapes of the allowed-key set of this half tile.
+      const bool w_none = __all_sync(0xffffffffu, (bits[0] | bits[1]) == 0u);
+      const bool w_all = __all_sync(0xffffffffu, (bits[0] & bits[1]) == 0xffffffffu);
+      const int shape = warp_direct ? 3 : (w_none ? 1 : (w_all ? 2 : 0));
       float sF0 = 0.0f, sF1 = 0.0f, sX0 = 0.0f, sX1 = 0.0f;
 #pragma unroll
       for (int ch = 0; ch < kHalf / 32; ++ch) {
         uint32_t pkF[16], pkX[16];
+        if (shape == 1) {  // no allowed key in this half for the whole warp
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = ch * 32 + 2 * i;
-          float y0, y1;
-          ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
-          const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
-          const bool in0 = (bits[ch] >> (2 * i)) & 1u;
-          const bool in1 = (bits[ch] >> (2 * i + 1)) & 1u;
-          float g0 = in0 ? f0 * kX : 0.0f;
-          float g1 = in1 ? f1 * kX : 0.0f;
-          if (warp_direct && direct) {
-            g0 = in0 ? fast_exp2(fmaf(u2f(sr[c0]), p.scale_log2, -uX)) : 0.0f;
-            g1 = in1 ? fast_exp2(fmaf(u2f(sr[c0 + 1]), p.scale_log2, -uX)) : 0.0f;
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = ch * 32 + 2 * i;
+            float y0, y1;
+            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
+            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
+            fadd2(sF0, sF1, sF0, sF1, f0, f1);
+            pkF[i] = pack_bf16x2(f0, f1);
+            pkX[i] = 0u;
           }
-          fadd2(sF0, sF1, sF0, sF1, f0, f1);
-          fadd2(sX0, sX1, sX0, sX1, g0, g1);
-          pkF[i] = pack_bf16x2(f0, f1);
-          pkX[i] = pack_bf16x2(g0, g1);
+        } else if (shape == 2) {  // every key allowed for the whole warp
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = ch * 32 + 2 * i;
+            float y0, y1, g0, g1;
+            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
+            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
+            ffma2(g0, g1, f0, f1, kX, kX, 0.0f, 0.0f);
+            fadd2(sF0, sF1, sF0, sF1, f0, f1);
+            fadd2(sX0, sX1, sX0, sX1, g0, g1);
+            pkF[i] = pack_bf16x2(f0, f1);
+            pkX[i] = pack_bf16x2(g0, g1);
+          }
+        } else if (shape == 0) {  // general: per-key selection
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = ch * 32 + 2 * i;
+            float y0, y1;
+            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
+            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
+            const float g0 = ((bits[ch] >> (2 * i)) & 1u) ? f0 * kX : 0.0f;
+            const float g1 = ((bits[ch] >> (2 * i + 1)) & 1u) ? f1 * kX : 0.0f;
+            fadd2(sF0, sF1, sF0, sF1, f0, f1);
+            fadd2(sX0, sX1, sX0, sX1, g0, g1);
+            pkF[i] = pack_bf16x2(f0, f1);
+            pkX[i] = pack_bf16x2(g0, g1);
+          }
+        } else {  // some row's masked base is far below its full base
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = ch * 32 + 2 * i;
+            float y0, y1;
+            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
+            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
+            const bool in0 = (bits[ch] >> (2 * i)) & 1u;
+            const bool in1 = (bits[ch] >> (2 * i + 1)) & 1u;
+            float g0 = in0 ? f0 * kX : 0.0f;
+            float g1 = in1 ? f1 * kX : 0.0f;
+            if (direct) {
+              g0 = in0 ? fast_exp2(fmaf(u2f(sr[c0]), p.scale_log2, -uX)) : 0.0f;
+              g1 = in1 ? fast_exp2(fmaf(u2f(sr[c0 + 1]), p.scale_log2, -uX)) : 0.0f;
+            }
+            fadd2(sF0, sF1, sF0, sF1, f0, f1);
+            fadd2(sX0, sX1, sX0, sX1, g0, g1);
+            pkF[i] = pack_bf16x2(f0, f1);
+            pkX[i] = pack_bf16x2(g0, g1);
+          }
         }
         // keys k -> column k/2: this half's 64 keys fill 32 columns
         tmem_st_32x32b_x16(s_col + half * 32 + ch * 16, pkF);
