@@ -110,7 +110,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", ident], stdout=open(self.path, "w"),
+                 "-lms", "100", "-i", ident], stdout=open(self.path, "w"),
                 stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -268,7 +268,7 @@ def run_capture(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(SI.WORKLOADS))
@@ -377,31 +377,31 @@ def main():
     if st != svg.SVG_OK:
         raise RuntimeError(f"device status {st} bits {bits}")
 
-    # end to end through the public API: pinned host inputs -> device -> host result
+    # end to end through the public API: pinned host inputs -> device -> pinned
+    # host output, every step, with the copies of neighbouring steps overlapped
+    # with compute by the streamed executor (StreamedLayer)
     e2e = None
     if not args.no_e2e:
-        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        from video_dit_spatial_b200.layer import StreamedLayer
+        del layer, o
+        torch.cuda.empty_cache()
+        o_h = torch.empty((wl.B, wl.H, wl.N, wl.d), dtype=torch.bfloat16).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, rows_h))
         d2h = o_h.numel() * o_h.element_size()
-
-        def e2e_step():
-            q.copy_(qh, non_blocking=True)
-            k.copy_(kh, non_blocking=True)
-            v.copy_(vh, non_blocking=True)
-            rows.copy_(rows_h, non_blocking=True)
-            layer.forward(q, k, v, rows, o, rebuild_masks=True)
-            o_h.copy_(o, non_blocking=True)
-
-        e2e_step()
+        sl = StreamedLayer(g, wl.n_samples, dev)
+        reps = max(4, min(args.steps, 8))
+        for i in range(2):
+            sl.submit(i, qh, kh, vh, rows_h, o_h)
+        sl.synchronize()
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = max(2, min(args.steps, 5))
-        e0.record(stream)
-        for _ in range(reps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(sl.s_in)
+        for i in range(2, 2 + reps):
+            sl.submit(i, qh, kh, vh, rows_h, o_h)
+        e1.record(sl.s_out)
+        sl.synchronize()
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / reps
         if dist is not None:
@@ -425,9 +425,9 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         kinds = SI.planted_head_kinds(wl)
         heads = [kinds.index(0), kinds.index(1)]
-        secs, fl = oracle_sample(wl, 24, heads)
+        secs, fl = oracle_sample(wl, 96, heads)
         cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"fp64 oracle attention output of 24 query rows x 2 heads (one spatial, "
+               "sample": f"fp64 oracle attention output of 96 query rows x 2 heads (one spatial, "
                          f"one temporal) of {wl.name}, with their block-mask rows",
                "seconds": secs}
 

@@ -78,3 +78,31 @@ def test_out_of_range_column_is_flagged_and_skipped(svg):
     # the valid block of row 0 still gives softmax(0) . 1 = 1
     assert torch.allclose(o.float(), torch.ones_like(o, dtype=torch.float32))
     status_clean()
+
+
+def test_streamed_layer_matches_plain_layer(svg):
+    # Three different host-resident items through the copy/compute pipeline must
+    # give exactly what the plain layer gives item by item (same kernels).
+    from video_dit_spatial_b200.layer import SparseVideoGenLayer, StreamedLayer
+    base = SI.TINY.replace(name="stream", d=128, T=5, P=300, n_text=77, H=4, n_spatial=2,
+                           n_samples_fixed=300, spatial_band=1, temporal_width=20,
+                           block_q=128, block_k=128)
+    g = svg.Geom.from_workload(base)
+    items = []
+    for i in range(3):
+        wl = base.replace(seed=5000 + i)
+        q, k, v = (t.pin_memory() for t in SI.make_qkv(wl))
+        rows = SI.sample_rows(wl).pin_memory()
+        o_h = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        items.append((q, k, v, rows, o_h))
+    sl = StreamedLayer(g, base.n_samples)
+    for i, it in enumerate(items):
+        sl.submit(i, *it)
+    sl.synchronize()
+    plain = SparseVideoGenLayer(g, base.n_samples)
+    for q, k, v, rows, o_h in items:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+        plain.forward(q.cuda(), k.cuda(), v.cuda(), rows.cuda(), o)
+        torch.cuda.synchronize()
+        assert torch.equal(o.cpu().view(torch.int16), o_h.view(torch.int16))
+    status_clean()

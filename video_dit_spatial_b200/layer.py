@@ -86,3 +86,60 @@ class SparseVideoGenLayer:
         dm = self.dense_mask
         svg_sparse_attention(self.geom, q, k, v, None, None, None, None, dm.row_ptr, dm.col_idx,
                              None, None, o, None, lse, stream=stream)
+
+
+class StreamedLayer:
+    """The layer over a sequence of host-resident inputs, with copies overlapped.
+
+    Each item is (q, k, v, sample_idx) in pinned host memory and an output
+    buffer o in pinned host memory. Three CUDA streams form a pipeline over
+    `depth` device buffer sets: while item i computes, the inputs of item i+1
+    are copied in and the output of item i-1 is copied out. All compute of
+    every item runs on one stream, so the layer's shared scratch (permuted
+    tensors, labels, workspace, masks) is used by one item at a time.
+    """
+
+    def __init__(self, geom: Geom, n_samples: int, device="cuda", depth: int = 2):
+        self.layer = SparseVideoGenLayer(geom, n_samples, device)
+        dev = self.layer.device
+        shape = (geom.B, geom.H, geom.N, geom.head_dim)
+        self.depth = depth
+        self.qkv = [tuple(torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
+                    for _ in range(depth)]
+        self.rows = [torch.empty(n_samples, dtype=torch.int32, device=dev) for _ in range(depth)]
+        self.out = [torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(depth)]
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_compute = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        mk = lambda: [torch.cuda.Event() for _ in range(depth)]  # noqa: E731
+        self.ev_in, self.ev_done, self.ev_out = mk(), mk(), mk()
+        self.started = [False] * depth
+        with torch.cuda.stream(self.s_compute):
+            self.layer.build_masks(stream=self.s_compute)
+
+    def submit(self, i: int, q_h, k_h, v_h, rows_h, o_h) -> None:
+        """Enqueues item number i (the caller numbers items 0, 1, 2, ...)."""
+        b = i % self.depth
+        q, k, v = self.qkv[b]
+        if self.started[b]:
+            self.s_in.wait_event(self.ev_done[b])  # inputs of the previous user computed
+        with torch.cuda.stream(self.s_in):
+            q.copy_(q_h, non_blocking=True)
+            k.copy_(k_h, non_blocking=True)
+            v.copy_(v_h, non_blocking=True)
+            self.rows[b].copy_(rows_h, non_blocking=True)
+            self.ev_in[b].record(self.s_in)
+        self.s_compute.wait_event(self.ev_in[b])
+        if self.started[b]:
+            self.s_compute.wait_event(self.ev_out[b])  # output buffer copied out
+        self.layer.forward(q, k, v, self.rows[b], self.out[b], stream=self.s_compute)
+        self.ev_done[b].record(self.s_compute)
+        self.s_out.wait_event(self.ev_done[b])
+        with torch.cuda.stream(self.s_out):
+            o_h.copy_(self.out[b], non_blocking=True)
+            self.ev_out[b].record(self.s_out)
+        self.started[b] = True
+
+    def synchronize(self) -> None:
+        for s in (self.s_in, self.s_compute, self.s_out):
+            s.synchronize()
