@@ -76,6 +76,20 @@ def _dist_env():
     return world, rank, local
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest value over all ranks (every rank takes the same collective)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------------------
 # algorithmic work
 # ---------------------------------------------------------------------------
@@ -340,11 +354,7 @@ def main():
     if dist is not None:
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
-    ms = ev0.elapsed_time(ev1) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
     gpu_launches = 7 * args.steps  # profile, finalize, 2 masks, permute_qkv, attention, unpermute
 
     # per-kernel timing (events on the launch stream), then the dense baseline
@@ -403,12 +413,8 @@ def main():
         e1.record(sl.s_out)
         sl.synchronize()
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / reps
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * attn_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / reps, dist, dev)
+        e2e = {"value": job_throughput(attn_flops, world, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     pk = _peaks()
@@ -433,7 +439,7 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": world * attn_flops / (ms * 1e-3) / 1e12, "unit": UNIT,
+            "metric": METRIC, "value": job_throughput(attn_flops, world, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
