@@ -239,6 +239,15 @@ svg_status svg_get_device_status(svg_stream_t stream, int32_t* bits);
  */
 svg_status svg_selftest_wait_timeout(int64_t limit_cycles, svg_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * svg_selftest_exp2 -- applies the kernels' FMA-pipe 2^y evaluation (range
+ * reduction to y = n + f, minimax cubic for 2^f, exponent-field scaling) to
+ * in[0..n) and writes out[0..n); device float arrays, n in [1, 2^31]. Lets a
+ * test bound its error against exact 2^y. Inputs below -125 are clamped to
+ * -125 (the result is then a value in (0, 2^-124]).
+ */
+svg_status svg_selftest_exp2(const float* in, float* out, int64_t n, svg_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* svg_status_string(svg_status status);
 

@@ -371,11 +371,34 @@ __global__ void wait_selftest_kernel(long long limit, int* status) {
 }
 }  // namespace
 
+__global__ void exp2_selftest_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                     int64_t n) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    exp2_poly2(out[i], out[i + 1], in[i], in[i + 1]);
+  } else if (i < n) {
+    float dummy;
+    exp2_poly2(out[i], dummy, in[i], 0.0f);
+  }
+}
+
 cudaError_t launch_wait_selftest(long long limit_cycles, int* status, cudaStream_t stream) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_cycles, status);
   return cudaGetLastError();
 }
 }  // namespace svg
+
+extern "C" svg_status svg_selftest_exp2(const float* in, float* out, int64_t n,
+                                        svg_stream_t stream) {
+  if (in == nullptr || out == nullptr || n < 1 || n > (static_cast<int64_t>(1) << 31))
+    return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  const int64_t pairs = (n + 1) / 2;
+  svg::exp2_selftest_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0,
+                              static_cast<cudaStream_t>(stream)>>>(in, out, n);
+  return cudaGetLastError() == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
+}
 
 extern "C" svg_status svg_selftest_wait_timeout(int64_t limit_cycles, svg_stream_t stream) {
   if (limit_cycles < 1 || limit_cycles > (static_cast<int64_t>(1) << 31)) return SVG_ERR_INVALID_ARG;
