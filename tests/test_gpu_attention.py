@@ -123,7 +123,7 @@ def test_empty_csr_rows_give_zero(svg):
     status_clean()
 
 
-FULL = [SI.COGVIDEOX, SI.HUNYUAN, SI.LONG]
+FULL = [SI.COGVIDEOX, SI.HUNYUAN, SI.LONG] + SI.sweep_workloads()
 
 
 @pytest.mark.parametrize("wl", FULL, ids=lambda w: w.name)

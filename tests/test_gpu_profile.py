@@ -86,7 +86,8 @@ def test_profile_unstructured_inputs(svg):
     status_clean()
 
 
-@pytest.mark.parametrize("wl", [SI.COGVIDEOX, SI.HUNYUAN], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [SI.COGVIDEOX, SI.HUNYUAN, SI.LONG, SI.sweep_workloads()[2]],
+                         ids=lambda w: w.name)
 def test_profile_full_size(svg, wl):
     q, k, v = SI.make_qkv(wl)
     rows = SI.sample_rows(wl)
@@ -95,7 +96,10 @@ def test_profile_full_size(svg, wl):
     assert list(labels) == kinds * wl.B
     sp = [h for h in range(wl.H) if kinds[h] == 0][:2]
     tp = [h for h in range(wl.H) if kinds[h] == 1][:2]
-    assert _check_heads(wl, q, k, v, rows, labels, mse, [(0, h) for h in sp + tp]) == 4
+    heads = [(0, h) for h in sp + tp]
+    if wl.B > 1:  # one head per label in the first and the last sample of the batch
+        heads = [(0, sp[0]), (0, tp[0]), (wl.B - 1, sp[0]), (wl.B - 1, tp[0])]
+    assert _check_heads(wl, q, k, v, rows, labels, mse, heads) == len(heads)
     status_clean()
 
 

@@ -349,10 +349,8 @@ namespace svg {
 namespace {
 __global__ void wait_selftest_kernel(long long limit, int* status) {
   __shared__ uint64_t never;
-  __shared__ int abort_flag;
   if (threadIdx.x == 0) {
     mbar_init(&never, 1);
-    abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -361,7 +359,6 @@ __global__ void wait_selftest_kernel(long long limit, int* status) {
     const long long t0 = clock64();
     while (!mbar_try_wait(&never, 0)) {
       if (clock64() - t0 > limit) {
-        abort_flag = 1;
         atomicOr(status, kDevErrTimeout);
         break;
       }

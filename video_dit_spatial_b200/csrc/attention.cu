@@ -387,6 +387,7 @@ constexpr int kPairMmaWarp = 9;
 // on the HunyuanVideo-shaped layer: 1 in 4 made the kernel slower (28.2 ->
 // 33.5 ms): the softmax is bound by its per-tile critical path, not by MUFU.
 constexpr int kPairEmuEvery = 0;
+[[maybe_unused]] constexpr int kEmuMod = kPairEmuEvery > 0 ? kPairEmuEvery : 1;
 constexpr int kPairLaunchRegs = 168;   // per thread at launch (3 warps per sub-partition)
 constexpr int kPairSoftmaxRegs = 224;  // softmax warpgroups after setmaxnreg.inc
 constexpr int kPairOtherRegs = 56;     // producer / MMA warpgroup after setmaxnreg.dec
@@ -716,7 +717,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       float s0 = 0.0f, s1 = 0.0f;
       // Full tiles may evaluate one pair in kPairEmuEvery on the FMA pipe; the
       // ragged tile uses MUFU only.
-      const bool full_tile = kvalid == BK;
+      [[maybe_unused]] const bool full_tile = kvalid == BK;
 #pragma unroll
       for (int ch = 0; ch < BK / 32; ++ch) {
         uint32_t pk[16];
@@ -726,7 +727,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           float y0, y1, e0, e1;
           ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -m_use, -m_use);
           bool emulate = false;
-          if constexpr (kPairEmuEvery > 0) emulate = full_tile && i % kPairEmuEvery == kPairEmuEvery - 1;
+          if constexpr (kPairEmuEvery > 0) emulate = full_tile && i % kEmuMod == kEmuMod - 1;
           if (emulate) {
             exp2_poly2(e0, e1, y0, y1);
           } else {

@@ -113,9 +113,11 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  // Launch order: every temporal-mask CTA (the slower kind: its allowed keys
+  // reach every frame) before any spatial-mask CTA, heads in order.
   const int tile = blockIdx.x;
-  const int X = blockIdx.y;  // 0: spatial mask, 1: temporal mask
-  const int bh = blockIdx.z;
+  const int bh = blockIdx.y;
+  const int X = 1 - static_cast<int>(blockIdx.z);  // 0: spatial mask, 1: temporal mask
   const int n = p.nkt;
 
   if (warp == 0) {
@@ -576,7 +578,7 @@ cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, flo
   auto kern = profile_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(pp.n_tiles, 2, d.BH), kThreads, C::kSmem, stream>>>(pp);
+  kern<<<dim3(pp.n_tiles, d.BH, 2), kThreads, C::kSmem, stream>>>(pp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float inv = 1.0f / (static_cast<float>(pp.n_samples) * static_cast<float>(D));
