@@ -248,20 +248,31 @@ def run_capture(args, wl):
     g = svg.Geom.from_workload(wl)
     q, k, v = (t.cuda() for t in SI.make_qkv(wl))
     rows = SI.sample_rows(wl).cuda()
-    layer = SparseVideoGenLayer(g, wl.n_samples)
+    layers = {name: SparseVideoGenLayer(g, wl.n_samples, layout=name)
+              for name in ("explicit", "fused", "gathered")}
+    labels = torch.tensor(SI.planted_head_kinds(wl) * wl.B, dtype=torch.int8)
+    for layer in layers.values():
+        layer.build_masks()
+        layer.labels.copy_(labels)
+    ex, fu, ga = layers["explicit"], layers["fused"], layers["gathered"]
     o = torch.empty_like(q)
-    layer.build_masks()
-    layer.labels.copy_(torch.tensor(SI.planted_head_kinds(wl) * wl.B, dtype=torch.int8))
-    if args.capture == "attention":
-        svg.svg_permute_qkv(g, q, k, v, layer.qp, layer.kp, layer.vp, layer.labels)
+    svg.svg_permute_qkv(g, q, k, v, ex.qp, ex.kp, ex.vp, ex.labels)
+    svg.svg_permute_qkv(g, None, k, v, None, fu.kp, fu.vp, fu.labels)
+
+    def fused_attention(layer, kp, vp):
+        m = layer.masks
+        return lambda: svg.svg_sparse_attention_fused(
+            g, q, k, v, kp, vp, layer.labels, m[0].row_ptr, m[0].col_idx, m[1].row_ptr,
+            m[1].col_idx, o)
     fns = {
-        "attention": lambda: svg.svg_sparse_attention(
-            g, q, k, v, layer.qp, layer.kp, layer.vp, layer.labels,
-            layer.masks[0].row_ptr, layer.masks[0].col_idx, layer.masks[1].row_ptr,
-            layer.masks[1].col_idx, o, layer.op),
-        "profile": lambda: layer.profile(q, k, v, rows),
-        "permute": lambda: svg.svg_permute_qkv(g, q, k, v, layer.qp, layer.kp, layer.vp,
-                                               layer.labels),
+        # the attention kernel of the default (fused) layout
+        "attention": fused_attention(fu, fu.kp, fu.vp),
+        "attention_gathered": fused_attention(ga, None, None),
+        "attention_explicit": lambda: svg.svg_sparse_attention(
+            g, q, k, v, ex.qp, ex.kp, ex.vp, ex.labels, ex.masks[0].row_ptr,
+            ex.masks[0].col_idx, ex.masks[1].row_ptr, ex.masks[1].col_idx, o, ex.op),
+        "profile": lambda: fu.profile(q, k, v, rows),
+        "permute": lambda: svg.svg_permute_qkv(g, q, k, v, ex.qp, ex.kp, ex.vp, ex.labels),
     }
     fn = fns[args.capture]
     for it in range(3):
@@ -289,7 +300,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--capture", choices=["attention", "profile", "permute"],
+    ap.add_argument("--capture", choices=["attention", "attention_gathered", "attention_explicit",
+                                          "profile", "permute"],
                     help="small case for an ncu capture: run one kernel 3 times on the "
                          "workload with --heads heads, print per-launch ms, no JSON line")
     ap.add_argument("--heads", type=int, default=4)
@@ -326,6 +338,7 @@ def main():
     rows = rows_h.to(dev)
     o = torch.empty_like(q)
     layer = SparseVideoGenLayer(g, wl.n_samples, dev)
+    layout = layer.layout
     stream = torch.cuda.current_stream()
 
     def step():
@@ -355,7 +368,9 @@ def main():
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
-    gpu_launches = 7 * args.steps  # profile, finalize, 2 masks, permute_qkv, attention, unpermute
+    # profile, finalize, 2 masks, attention, plus the layout passes: permute_qkv and
+    # unpermute (explicit), permute of K and V (fused), none (gathered)
+    gpu_launches = {"explicit": 7, "fused": 6, "gathered": 5}[layout] * args.steps
 
     # per-kernel timing (events on the launch stream), then the dense baseline
     def time_fn(fn, reps):
@@ -371,13 +386,37 @@ def main():
 
     ms_profile = time_fn(lambda: layer.profile(q, k, v, rows), 5)
     ms_masks = time_fn(layer.build_masks, 5)
-    ms_permute = time_fn(lambda: svg.svg_permute_qkv(g, q, k, v, layer.qp, layer.kp, layer.vp,
-                                                     layer.labels), 5)
-    ms_unpermute = time_fn(lambda: svg.svg_unpermute(g, layer.op, o, layer.labels), 5)
-    ms_attn = time_fn(lambda: svg.svg_sparse_attention(
-        g, q, k, v, layer.qp, layer.kp, layer.vp, layer.labels,
-        layer.masks[0].row_ptr, layer.masks[0].col_idx, layer.masks[1].row_ptr,
-        layer.masks[1].col_idx, o, layer.op), max(3, args.steps))
+    # the attention kernel alone on the layer's layout (the roofline's kernel),
+    # and each way of doing the layout transformation, for comparison
+    m = layer.masks
+    labels_d = layer.labels
+
+    def attn_fused(kp, vp):
+        return lambda: svg.svg_sparse_attention_fused(
+            g, q, k, v, kp, vp, labels_d, m[0].row_ptr, m[0].col_idx, m[1].row_ptr,
+            m[1].col_idx, o)
+    kp, vp = (torch.empty_like(q) for _ in range(2))
+    ms_permute_kv = time_fn(lambda: svg.svg_permute_qkv(g, None, k, v, None, kp, vp, labels_d),
+                            5)
+    ms_attn_fused = time_fn(attn_fused(kp, vp), max(3, args.steps))
+    ms_attn_gathered = time_fn(attn_fused(None, None), 3)
+    qp, op = (torch.empty_like(q) for _ in range(2))
+    ms_permute = time_fn(lambda: svg.svg_permute_qkv(g, q, k, v, qp, kp, vp, labels_d), 5)
+    ms_unpermute = time_fn(lambda: svg.svg_unpermute(g, op, o, labels_d), 5)
+    ms_attn_explicit = time_fn(lambda: svg.svg_sparse_attention(
+        g, q, k, v, qp, kp, vp, labels_d, m[0].row_ptr, m[0].col_idx, m[1].row_ptr,
+        m[1].col_idx, o, op), max(3, args.steps // 2))
+    del kp, vp, qp, op
+    torch.cuda.empty_cache()
+    layouts_ms = {
+        "explicit": {"permute_qkv": ms_permute, "attention": ms_attn_explicit,
+                     "unpermute": ms_unpermute,
+                     "total": ms_permute + ms_attn_explicit + ms_unpermute},
+        "fused": {"permute_kv": ms_permute_kv, "attention": ms_attn_fused,
+                  "total": ms_permute_kv + ms_attn_fused},
+        "gathered": {"attention": ms_attn_gathered, "total": ms_attn_gathered},
+    }
+    ms_attn = layouts_ms[layout]["attention"]
     ms_dense = None
     if not args.no_dense:
         od = torch.empty_like(q)
@@ -419,7 +458,7 @@ def main():
 
     pk = _peaks()
     achieved = attn_flops / (ms_attn * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "sparse_attention_kernel", "achieved": achieved,
+    roofline = {"bound": "tensor", "kernel": "sparse_attention_pair_kernel", "achieved": achieved,
                 "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / pk["bf16_tflops_sustained"],
                 "peak_kind": f"bf16 dense, sustained, {pk['source']}",
@@ -455,9 +494,10 @@ def main():
             "layer_speedup_vs_dense": (ms_dense / ms) if ms_dense else None,
             "attn_tflops": achieved,
             "dense_tflops": (dense_flops / (ms_dense * 1e-3) / 1e12) if ms_dense else None,
-            "kernel_ms": {"profile": ms_profile, "block_masks": ms_masks,
-                          "permute_qkv": ms_permute, "attention": ms_attn,
-                          "unpermute": ms_unpermute},
+            "layout": layout,
+            "kernel_ms": dict({"profile": ms_profile, "block_masks": ms_masks},
+                              **{k: t for k, t in layouts_ms[layout].items() if k != "total"}),
+            "layouts_ms": layouts_ms,
             "labels_temporal": int(np.sum(labels == 1)),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": gpu_launches, "clocks": clock_info,

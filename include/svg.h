@@ -183,7 +183,9 @@ svg_status svg_permute(const svg_geom* geom, const svg_bf16* in, svg_bf16* out,
 svg_status svg_unpermute(const svg_geom* geom, const svg_bf16* in, svg_bf16* out,
                          const int8_t* labels, svg_stream_t stream);
 
-/* svg_permute_qkv -- svg_permute of Q, K and V in one launch. */
+/* svg_permute_qkv -- svg_permute of Q, K and V in one launch. q and qp may
+ * both be NULL: then only K and V are permuted (the input of
+ * svg_sparse_attention_fused with position-major K/V copies). */
 svg_status svg_permute_qkv(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
                            const svg_bf16* v, svg_bf16* qp, svg_bf16* kp, svg_bf16* vp,
                            const int8_t* labels, svg_stream_t stream);
@@ -219,6 +221,44 @@ svg_status svg_sparse_attention(const svg_geom* geom, const svg_bf16* q, const s
                                 const int32_t* row_ptr_s, const int32_t* col_idx_s,
                                 const int32_t* row_ptr_t, const int32_t* col_idx_t,
                                 svg_bf16* o, svg_bf16* op, float* lse, svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * svg_sparse_attention_fused -- svg_sparse_attention with the layout
+ * transformation folded into the attention kernel (SVG abstract: the
+ * "hardware-efficient tensor layout transformation"): no permuted copy of Q
+ * or O is written, and optionally none of K and V either.
+ * Every head reads q in frame-major order. A head labelled temporal still
+ * attends in position-major order over the temporal CSR: its query tiles are
+ * assembled row by row in that order (TMA tile::gather4 row gathers,
+ * frame-major row pi^-1(j) for position-major row j) and each output row is
+ * stored at its frame-major place. Its key/value tiles come either from
+ * position-major copies kp, vp (plain tiled loads) or, with kp = vp = NULL,
+ * are gathered row by row from k, v like the queries (no copy at all, but
+ * row gathers move far fewer bytes per cycle than tiled loads, so this form is
+ * slower on long key lists). The result equals
+ *   svg_permute_qkv -> svg_sparse_attention -> svg_unpermute
+ * bit for bit (same arithmetic in the same order), with lse, if given, also
+ * in frame-major rows.
+ *   q,k,v,o        device bf16 [B,H,N,d], frame-major, every head.
+ *   kp,vp          device bf16 [B,H,N,d], position-major copies of k and v
+ *                  for the temporal heads (svg_permute_qkv with q = qp =
+ *                  NULL), or both NULL.
+ *   labels         device int8 [B*H] (required).
+ *   row_ptr_s, col_idx_s, row_ptr_t, col_idx_t  device CSR of both masks
+ *                  (required), as for svg_sparse_attention.
+ *   lse            device float [B,H,N] out (frame-major rows) or NULL.
+ * Errors: INVALID_ARG (NULL or misaligned pointer, only one of kp/vp, bad
+ *   geometry),
+ *   UNSUPPORTED (block_q != 128, B*H*N >= 2^31 rows, or a device where the
+ *   paired-tile kernel cannot run), CUDA.
+ */
+svg_status svg_sparse_attention_fused(const svg_geom* geom, const svg_bf16* q,
+                                      const svg_bf16* k, const svg_bf16* v,
+                                      const svg_bf16* kp, const svg_bf16* vp,
+                                      const int8_t* labels, const int32_t* row_ptr_s,
+                                      const int32_t* col_idx_s, const int32_t* row_ptr_t,
+                                      const int32_t* col_idx_t, svg_bf16* o, float* lse,
+                                      svg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * svg_get_device_status -- synchronises `stream`, then reads and clears the

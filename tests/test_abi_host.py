@@ -102,6 +102,27 @@ def test_invalid_arguments_are_rejected_before_launch(svg):
     assert lib.svg_sparse_attention(ctypes.byref(g), 256, 256, 256, 256, None, None, None,
                                     256, 256, 256, 256, 256, None, None, None) == \
         svg.SVG_ERR_INVALID_ARG
+    # fused layout path: labels and both CSRs required; kp/vp both or neither;
+    # 128-row query blocks only
+    f = lib.svg_sparse_attention_fused
+    g128 = _geom(svg, bq=128)
+    assert f(ctypes.byref(g128), 256, 256, 256, None, None, None, 256, 256, 256, 256, 256,
+             None, None) == svg.SVG_ERR_INVALID_ARG
+    assert f(ctypes.byref(g128), 256, 256, 256, None, None, 256, 256, 256, None, 256, 256,
+             None, None) == svg.SVG_ERR_INVALID_ARG
+    assert f(ctypes.byref(g128), 256, 264, 256, None, None, 256, 256, 256, 256, 256, 256,
+             None, None) == svg.SVG_ERR_INVALID_ARG
+    assert f(ctypes.byref(g128), 256, 256, 256, 256, None, 256, 256, 256, 256, 256, 256,
+             None, None) == svg.SVG_ERR_INVALID_ARG
+    g64 = _geom(svg, bq=64)
+    assert f(ctypes.byref(g64), 256, 256, 256, None, None, 256, 256, 256, 256, 256, 256,
+             None, None) == svg.SVG_ERR_UNSUPPORTED
+    huge = _geom(svg, bq=128, T=1 << 15, P=1 << 14, B=1, H=4)  # 4 * 2^29 rows >= 2^31
+    assert f(ctypes.byref(huge), 256, 256, 256, None, None, 256, 256, 256, 256, 256, 256,
+             None, None) == svg.SVG_ERR_UNSUPPORTED
+    # permute of K and V only: q and qp both NULL or both given
+    assert lib.svg_permute_qkv(ctypes.byref(g), 256, 4096, 8192, None, 1 << 20, 1 << 21,
+                               None, None) == svg.SVG_ERR_INVALID_ARG
     # overlapping permute buffers
     assert lib.svg_permute(ctypes.byref(g), 4096, 4096 + 256, None, None) == \
         svg.SVG_ERR_INVALID_ARG

@@ -22,8 +22,10 @@ def svg():
 
 
 def _layer(svg, g, n_samples=16):
+    # the explicit layout path (permute -> attention -> unpermute); the fused
+    # path is compared with it in test_gpu_fused_layout.py
     from video_dit_spatial_b200.layer import SparseVideoGenLayer
-    return SparseVideoGenLayer(g, n_samples)
+    return SparseVideoGenLayer(g, n_samples, layout="explicit")
 
 
 # T, P, L, d, bq, bk, s, w, B, H

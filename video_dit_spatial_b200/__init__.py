@@ -35,7 +35,7 @@ STATUS_NAMES = {0: "SVG_OK", 1: "SVG_ERR_INVALID_ARG", 2: "SVG_ERR_UNSUPPORTED",
 EXPORTED = [
     "svg_mask_nnz", "svg_build_block_mask", "svg_profile_workspace_bytes",
     "svg_profile_heads", "svg_profile_heads_noalloc", "svg_permute", "svg_unpermute", "svg_permute_qkv",
-    "svg_sparse_attention", "svg_get_device_status", "svg_selftest_wait_timeout",
+    "svg_sparse_attention", "svg_sparse_attention_fused", "svg_get_device_status", "svg_selftest_wait_timeout",
     "svg_selftest_exp2",
     "svg_status_string", "svg_version",
 ]
@@ -101,6 +101,7 @@ def load() -> ctypes.CDLL:
         "svg_unpermute": [_c_geom_p, _vp, _vp, _vp, _vp],
         "svg_permute_qkv": [_c_geom_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
         "svg_sparse_attention": [_c_geom_p] + [_vp] * 15,
+        "svg_sparse_attention_fused": [_c_geom_p] + [_vp] * 13,
         "svg_get_device_status": [_vp, ctypes.POINTER(_i32)],
         "svg_selftest_wait_timeout": [_i64, _vp],
         "svg_selftest_exp2": [_vp, _vp, _i64, _vp],
@@ -207,6 +208,15 @@ def svg_sparse_attention(geom: Geom, q, k, v, qp, kp, vp, labels, row_ptr_s, col
         ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp),
         _ptr(labels), _ptr(row_ptr_s), _ptr(col_idx_s), _ptr(row_ptr_t), _ptr(col_idx_t),
         _ptr(o), _ptr(op), _ptr(lse), _stream(stream)))
+
+
+def svg_sparse_attention_fused(geom: Geom, q, k, v, kp, vp, labels, row_ptr_s, col_idx_s,
+                               row_ptr_t, col_idx_t, o, lse=None, stream=None) -> None:
+    _check("svg_sparse_attention_fused", load().svg_sparse_attention_fused(
+        ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(kp), _ptr(vp), _ptr(labels),
+        _ptr(row_ptr_s),
+        _ptr(col_idx_s), _ptr(row_ptr_t), _ptr(col_idx_t), _ptr(o), _ptr(lse),
+        _stream(stream)))
 
 
 def svg_get_device_status(stream=None):

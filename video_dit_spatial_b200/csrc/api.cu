@@ -145,6 +145,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int32_t d, int32_t N, in
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_rows_bf16(CUtensorMap* map, const void* base, int32_t d, int64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64u, 1u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace svg
 
 using svg::Dims;
@@ -289,6 +303,12 @@ svg_status svg_unpermute(const svg_geom* geom, const svg_bf16* in, svg_bf16* out
 svg_status svg_permute_qkv(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
                            const svg_bf16* v, svg_bf16* qp, svg_bf16* kp, svg_bf16* vp,
                            const int8_t* labels, svg_stream_t stream) {
+  if ((q == nullptr) != (qp == nullptr)) return SVG_ERR_INVALID_ARG;
+  if (q == nullptr) {  // K and V only
+    const svg_bf16* i[2] = {k, v};
+    svg_bf16* o[2] = {kp, vp};
+    return permute_common(geom, 2, i, o, labels, false, stream);
+  }
   const svg_bf16* i[3] = {q, k, v};
   svg_bf16* o[3] = {qp, kp, vp};
   return permute_common(geom, 3, i, o, labels, false, stream);
@@ -318,11 +338,45 @@ svg_status svg_sparse_attention(const svg_geom* geom, const svg_bf16* q, const s
   int* status = svg::device_status_word(&err);
   if (status == nullptr) return SVG_ERR_CUDA;
   svg::AttnArgs a{q, k, v, qp, kp, vp, labels, row_ptr_s, col_idx_s, row_ptr_t, col_idx_t,
-                  o, op, lse};
+                  o, op, lse, false};
   if (svg::launch_sparse_attention(d, a, status, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return SVG_ERR_CUDA;
   return SVG_OK;
+}
+
+svg_status svg_sparse_attention_fused(const svg_geom* geom, const svg_bf16* q,
+                                      const svg_bf16* k, const svg_bf16* v,
+                                      const svg_bf16* kp, const svg_bf16* vp,
+                                      const int8_t* labels, const int32_t* row_ptr_s,
+                                      const int32_t* col_idx_s, const int32_t* row_ptr_t,
+                                      const int32_t* col_idx_t, svg_bf16* o, float* lse,
+                                      svg_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || labels == nullptr ||
+      row_ptr_s == nullptr || col_idx_s == nullptr || row_ptr_t == nullptr ||
+      col_idx_t == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  if (!svg::aligned16(q) || !svg::aligned16(k) || !svg::aligned16(v) || !svg::aligned16(o))
+    return SVG_ERR_INVALID_ARG;
+  if ((kp == nullptr) != (vp == nullptr)) return SVG_ERR_INVALID_ARG;
+  if (kp != nullptr && (!svg::aligned16(kp) || !svg::aligned16(vp))) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_geom(geom, true);
+  if (st != SVG_OK) return st;
+  if (geom->block_q != 128) return SVG_ERR_UNSUPPORTED;
+  // gather coordinates are signed 32-bit rows of the [B*H*N, d] view
+  const int64_t rows = static_cast<int64_t>(geom->B) * geom->H *
+                       (static_cast<int64_t>(geom->T) * geom->P + geom->n_text);
+  if (rows > 0x7fffffffLL) return SVG_ERR_UNSUPPORTED;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  svg::AttnArgs a{q, k, v, nullptr, kp, vp, labels, row_ptr_s, col_idx_s,
+                  row_ptr_t, col_idx_t, o, nullptr, lse, true};
+  err = svg::launch_sparse_attention(d, a, status, static_cast<cudaStream_t>(stream));
+  if (err == cudaErrorNotSupported) return SVG_ERR_UNSUPPORTED;
+  return err == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
 }
 
 svg_status svg_get_device_status(svg_stream_t stream, int32_t* bits) {

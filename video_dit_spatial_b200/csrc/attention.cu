@@ -61,6 +61,10 @@ struct Cfg {
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
 
+// Tensor maps [1] are the position-major copies (3-D tiled maps), or, with
+// `gather` set, a 2-D row map (box 64 x 1) over the frame-major q from which
+// temporal heads gather their query rows in position-major order; k and v
+// likewise with `gather_kv`, else tiled maps over position-major copies.
 struct __align__(64) AttnParams {
   CUtensorMap tm_q[2], tm_k[2], tm_v[2];  // [0]: frame-major, [1]: position-major
   const int8_t* labels;
@@ -71,11 +75,23 @@ struct __align__(64) AttnParams {
   int* status;
   int32_t N, Nv, BH, nqb, nkb, bq, bk;
   int32_t has_permuted;
+  int32_t gather, gather_kv, T, P;
   float scale_log2;
 };
 
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+// Frame-major row of position-major row j (the inverse of the layout
+// transformation pi(f*P + p) = p*T + f; text rows stay in place). Rows past
+// the end are clamped to the last row: they only fill the ragged tail of a
+// tile, whose keys the softmax masks and whose query rows are never stored.
+__device__ __forceinline__ int frame_major_row(int j, int N, int Nv, int T, int P) {
+  if (j >= N) j = N - 1;
+  if (j >= Nv) return j;
+  const int pos = j / T;
+  return (j - pos * T) * P + pos;
+}
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -480,10 +496,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   const int label = p.labels ? static_cast<int>(p.labels[bh]) : SVG_HEAD_SPATIAL;
   const int sel = label == SVG_HEAD_TEMPORAL ? 1 : 0;
-  if ((label != SVG_HEAD_SPATIAL && label != SVG_HEAD_TEMPORAL) || (sel == 1 && !p.has_permuted)) {
+  if ((label != SVG_HEAD_SPATIAL && label != SVG_HEAD_TEMPORAL) ||
+      (sel == 1 && !p.has_permuted && !p.gather)) {
     if (tid == 0) atomicOr(p.status, kDevErrBounds);
     return;
   }
+  // Temporal heads of the fused layout path: query rows gathered in
+  // position-major order from the frame-major q, outputs scattered back; key
+  // and value rows gathered too, or read from position-major copies.
+  const bool gather = p.gather != 0 && sel == 1;
+  const bool gather_kv = gather && p.gather_kv != 0;
   // CSR rows of the two tiles (tile B may not exist at an odd tail)
   int qb[2], nt[2];
   const int32_t* cols[2];
@@ -535,19 +557,44 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairOtherRegs));
     if (warp == kPairProducerWarp) {
       // ------------------------------------------------------------ producer
-      if (lane_id() == 0 && any_work) {
+      // Lane 0 waits and posts the byte counts. Tiled loads come from lane 0;
+      // row gathers (temporal heads of the fused layout path) from lanes
+      // 0..rows/4-1, four rows each per 64-column panel.
+      const int lane = lane_id();
+      if (any_work) {
         const CUtensorMap* mq = &p.tm_q[sel];
         const CUtensorMap* mk = &p.tm_k[sel];
         const CUtensorMap* mv = &p.tm_v[sel];
         const uint64_t keep = l2_policy_evict_last();
+        // Rows j0 .. j0+nrows-1 (position-major) of head bh -> dst, a tile of
+        // nrows x 128 B panels, panel stride `panel`.
+        auto gather_rows = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* b, int j0,
+                               int nrows, int panel, uint64_t policy) {
+          const int r = 4 * lane;
+          if (r >= nrows) return;
+          int src[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            src[i] = bh * p.N + frame_major_row(j0 + r + i, p.N, p.Nv, p.T, p.P);
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_gather4_hint(dst + pn * panel + r * 128, map, b, pn * 64, src[0], src[1], src[2],
+                             src[3], policy);
+        };
         uint32_t qbytes = 0;
         for (int t = 0; t < 2; ++t) qbytes += nt[t] > 0 ? C::kQBytes : 0;
-        mbar_arrive_expect_tx(&bar->q_full, qbytes);
-        for (int t = 0; t < 2; ++t)
-          if (nt[t] > 0)
+        if (lane == 0) mbar_arrive_expect_tx(&bar->q_full, qbytes);
+        __syncwarp();
+        for (int t = 0; t < 2; ++t) {
+          if (nt[t] == 0) continue;
+          if (gather) {
+            gather_rows(sQ + t * C::kQBytes, mq, &bar->q_full, qb[t] * 128, 128, C::kQPanel, keep);
+          } else if (lane == 0) {
             for (int pn = 0; pn < C::kPanels; ++pn)
               tma_load_3d(sQ + t * C::kQBytes + pn * C::kQPanel, mq, &bar->q_full, pn * 64,
                           qb[t] * 128, bh);
+          }
+        }
         UnionWalk walk{cols[0], cols[1], nt[0], nt[1]};
         int issued = 0;
         for (int u = 0;; ++u) {
@@ -557,23 +604,38 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (c < 0 || c >= p.nkb) c = 0;  // flagged and masked by the softmax warps
           const int st = u % C::kStages;
           const uint32_t par = ((u / C::kStages) & 1) ^ 1;
-          if (!mbar_wait(&bar->k_empty[st], par, abort_flag, p.status)) break;
-          mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kKVPanel, mk, &bar->k_full[st],
-                             pn * 64, c * BK, bh, keep);
-          if (!mbar_wait(&bar->v_empty[st], par, abort_flag, p.status)) {
+          bool ok = true;
+          if (lane == 0) {
+            ok = mbar_wait(&bar->k_empty[st], par, abort_flag, p.status);
+            if (ok) mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
+          }
+          if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+          if (gather_kv) {
+            gather_rows(sK + st * C::kKVBytes, mk, &bar->k_full[st], c * BK, BK, C::kKVPanel, keep);
+          } else if (lane == 0) {
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kKVPanel, mk, &bar->k_full[st],
+                               pn * 64, c * BK, bh, keep);
+          }
+          if (lane == 0) {
+            ok = mbar_wait(&bar->v_empty[st], par, abort_flag, p.status);
+            if (ok) mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
+          }
+          if (!__shfl_sync(0xffffffffu, ok, 0)) {
             issued = -(u + 1);  // K of step u is in flight, V is not
             break;
           }
-          mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kKVPanel, mv, &bar->v_full[st],
-                             pn * 64, c * BK, bh, keep);
+          if (gather_kv) {
+            gather_rows(sV + st * C::kKVBytes, mv, &bar->v_full[st], c * BK, BK, C::kKVPanel, keep);
+          } else if (lane == 0) {
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kKVPanel, mv, &bar->v_full[st],
+                               pn * 64, c * BK, bh, keep);
+          }
           issued = u + 1;
         }
-        if (*abort_flag) {
-          // Let every copy this thread started land before the CTA retires.
+        if (lane == 0 && *abort_flag) {
+          // Let every copy this warp started land before the CTA retires.
           const int done = issued < 0 ? -issued : issued;
           for (int u = (done > C::kStages ? done - C::kStages : 0); u < done; ++u) {
             const int st = u % C::kStages;
@@ -764,7 +826,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     if (ok && n > 0) ok = mbar_wait(&bar->o_final[t], 0, abort_flag, p.status);
     tc_fence_after();
     const bool have_o = __all_sync(0xffffffffu, ok) && n > 0;
-    svg_bf16* out = p.out[sel] + (static_cast<size_t>(bh) * p.N + row) * D;
+    // the fused layout path writes temporal rows straight to their frame-major place
+    const int out_row = gather && row_valid ? frame_major_row(row, p.N, p.Nv, p.T, p.P) : row;
+    svg_bf16* out = p.out[sel] + (static_cast<size_t>(bh) * p.N + out_row) * D;
     const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
 #pragma unroll
     for (int ch = 0; ch < D / 32; ++ch) {
@@ -786,7 +850,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
     }
     if (p.lse != nullptr && row_valid) {
-      p.lse[static_cast<size_t>(bh) * p.N + row] =
+      p.lse[static_cast<size_t>(bh) * p.N + out_row] =
           (have_o && l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
@@ -817,7 +881,11 @@ cudaError_t launch_pair(const Dims& d, const AttnParams& p, cudaStream_t stream)
   int resident = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kPairThreads, C::kSmem);
   if (e != cudaSuccess) return e;
-  if (fa.numRegs != kPairLaunchRegs || resident < 1) return launch_impl<D, BK>(d, p, stream);
+  if (fa.numRegs != kPairLaunchRegs || resident < 1) {
+    // the single-tile kernel has no row gathers
+    if (p.gather) return cudaErrorNotSupported;
+    return launch_impl<D, BK>(d, p, stream);
+  }
   dim3 grid(static_cast<unsigned>(((d.nqb + 1) / 2) * d.BH));
   kern<<<grid, kPairThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError();
@@ -840,12 +908,24 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
                                     cudaStream_t stream) {
   AttnParams p;
   memset(&p, 0, sizeof(p));
-  const bool perm = a.qp != nullptr;
+  const bool perm = a.qp != nullptr && !a.fused;
+  if (a.fused && d.bq != 128) return cudaErrorNotSupported;
   if (!make_tmap_bf16(&p.tm_q[0], a.q, d.d, d.N, d.BH, d.bq) ||
       !make_tmap_bf16(&p.tm_k[0], a.k, d.d, d.N, d.BH, d.bk) ||
       !make_tmap_bf16(&p.tm_v[0], a.v, d.d, d.N, d.BH, d.bk))
     return cudaErrorInvalidValue;
-  if (perm) {
+  if (a.fused) {
+    const int64_t rows = static_cast<int64_t>(d.BH) * d.N;
+    if (!make_tmap_rows_bf16(&p.tm_q[1], a.q, d.d, rows)) return cudaErrorInvalidValue;
+    if (a.kp != nullptr) {  // position-major copies of K and V
+      if (!make_tmap_bf16(&p.tm_k[1], a.kp, d.d, d.N, d.BH, d.bk) ||
+          !make_tmap_bf16(&p.tm_v[1], a.vp, d.d, d.N, d.BH, d.bk))
+        return cudaErrorInvalidValue;
+    } else if (!make_tmap_rows_bf16(&p.tm_k[1], a.k, d.d, rows) ||
+               !make_tmap_rows_bf16(&p.tm_v[1], a.v, d.d, rows)) {
+      return cudaErrorInvalidValue;
+    }
+  } else if (perm) {
     if (!make_tmap_bf16(&p.tm_q[1], a.qp, d.d, d.N, d.BH, d.bq) ||
         !make_tmap_bf16(&p.tm_k[1], a.kp, d.d, d.N, d.BH, d.bk) ||
         !make_tmap_bf16(&p.tm_v[1], a.vp, d.d, d.N, d.BH, d.bk))
@@ -861,7 +941,7 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
   p.row_ptr[1] = a.row_ptr_t ? a.row_ptr_t : a.row_ptr_s;
   p.col_idx[1] = a.col_idx_t ? a.col_idx_t : a.col_idx_s;
   p.out[0] = a.o;
-  p.out[1] = a.op ? a.op : a.o;
+  p.out[1] = a.op && !a.fused ? a.op : a.o;
   p.lse = a.lse;
   p.status = status;
   p.N = d.N;
@@ -872,6 +952,10 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
   p.bq = d.bq;
   p.bk = d.bk;
   p.has_permuted = perm && a.op != nullptr && a.row_ptr_t != nullptr && a.col_idx_t != nullptr;
+  p.gather = a.fused ? 1 : 0;
+  p.gather_kv = a.fused && a.kp == nullptr ? 1 : 0;
+  p.T = d.T;
+  p.P = d.P;
   p.scale_log2 = d.scale * 1.4426950408889634f;
   if (d.bq == 128) {
     if (d.d == 128 && d.bk == 128) return launch_pair<128, 128>(d, p, stream);

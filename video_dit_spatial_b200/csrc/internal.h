@@ -86,6 +86,9 @@ int* device_status_word(cudaError_t* err);
 // Tensor map of a [BH, N, d] bf16 tensor with a (64 x rows x 1) box, 128-byte swizzle.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int32_t d, int32_t N, int32_t BH,
                     int32_t box_rows);
+// Row map of the same tensor seen as [BH*N, d] with a 64 x 1 box, 128-byte
+// swizzle: the tensor map of tile::gather4 row gathers.
+bool make_tmap_rows_bf16(CUtensorMap* map, const void* base, int32_t d, int64_t rows);
 
 // Launchers (validated arguments; return the launch error).
 cudaError_t launch_permute(const Dims& d, int n_tensors, const svg_bf16* const* in,
@@ -100,6 +103,7 @@ struct AttnArgs {
   const int32_t *row_ptr_s, *col_idx_s, *row_ptr_t, *col_idx_t;
   svg_bf16 *o, *op;
   float* lse;
+  bool fused;  // temporal heads gather from q, k, v and scatter to o (qp..op unused)
 };
 cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* status,
                                     cudaStream_t stream);

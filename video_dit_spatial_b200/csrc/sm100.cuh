@@ -105,6 +105,22 @@ __device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// Row gather global -> shared (tile::gather4, 2-D tensor map whose box is 64
+// columns x 1 row): rows r0..r3 at column x land as four consecutive 128-byte
+// rows at smem_dst (which must be 512-byte aligned inside a 1024-byte aligned
+// tile, so the 128-byte swizzle matches the tiled loads). Completion counted on
+// `bar`, with an L2 eviction-priority hint.
+__device__ __forceinline__ void tma_gather4_hint(void* smem_dst, const CUtensorMap* map,
+                                                 uint64_t* bar, int x, int r0, int r1, int r2,
+                                                 int r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));

@@ -6,6 +6,16 @@ layout transformation); block-sparse attention runs over each head's block
 mask; temporal outputs are moved back. This class only owns device buffers
 (allocated with torch) and calls the library's entry points in that order on
 one stream; every step is a libsvg kernel.
+
+`layout` chooses how the layout transformation is done:
+  "explicit"  permute Q, K, V of temporal heads, attend, un-permute O;
+  "fused"     permute K, V only; the attention kernel gathers the query rows of
+              temporal heads in position-major order and stores each output row
+              at its frame-major place (no Q or O copies, no un-permute pass);
+  "gathered"  nothing is permuted: key/value rows are gathered in the kernel
+              too (least memory; row gathers are slower than tiled loads).
+"fused" and "gathered" need 128-row query blocks; they give the same bits as
+"explicit".
 """
 from __future__ import annotations
 
@@ -15,7 +25,7 @@ import torch
 
 from . import (Geom, SVG_MASK_DENSE, SVG_MASK_SPATIAL, SVG_MASK_TEMPORAL, svg_build_block_mask,
                svg_mask_nnz, svg_permute_qkv, svg_profile_heads, svg_profile_workspace_bytes,
-               svg_sparse_attention, svg_unpermute)
+               svg_sparse_attention, svg_sparse_attention_fused, svg_unpermute)
 
 
 class BlockMaskCSR:
@@ -31,9 +41,18 @@ class BlockMaskCSR:
         svg_build_block_mask(geom, self.kind, self.row_ptr, self.col_idx, stream=stream)
 
 
+LAYOUTS = ("explicit", "fused", "gathered")
+
+
 class SparseVideoGenLayer:
-    def __init__(self, geom: Geom, n_samples: int, device="cuda"):
+    def __init__(self, geom: Geom, n_samples: int, device="cuda",
+                 layout: Optional[str] = None):
         self.geom = geom
+        if layout is None:
+            layout = "fused" if geom.block_q == 128 else "explicit"
+        if layout not in LAYOUTS:
+            raise ValueError(f"layout must be one of {LAYOUTS}")
+        self.layout = layout
         self.n_samples = n_samples
         self.device = torch.device(device)
         B, H, N, d = geom.B, geom.H, geom.N, geom.head_dim
@@ -45,10 +64,12 @@ class SparseVideoGenLayer:
         self.workspace = torch.empty(max(wbytes // 4, 1), dtype=torch.float32, device=self.device)
         self.labels = torch.empty(B * H, dtype=torch.int8, device=self.device)
         self.mse = torch.empty(B * H * 2, dtype=torch.float32, device=self.device)
-        self.qp = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
-        self.kp = torch.empty_like(self.qp)
-        self.vp = torch.empty_like(self.qp)
-        self.op = torch.empty_like(self.qp)
+        self.qp = self.kp = self.vp = self.op = None
+        mk = lambda: torch.empty(shape, dtype=torch.bfloat16, device=self.device)  # noqa: E731
+        if layout == "explicit":
+            self.qp, self.op = mk(), mk()
+        if layout in ("explicit", "fused"):
+            self.kp, self.vp = mk(), mk()
         self.masks_built = False
 
     def build_masks(self, stream=None) -> None:
@@ -61,8 +82,20 @@ class SparseVideoGenLayer:
                           n_samples=self.n_samples, stream=stream)
 
     def attend(self, q, k, v, o, lse=None, stream=None) -> None:
-        """Permute temporal heads, block-sparse attention, un-permute (labels as set)."""
+        """Permute temporal heads, block-sparse attention, un-permute (labels as set).
+
+        lse, if given, is in frame-major rows on the fused layouts and in
+        each head's own layout on the explicit one.
+        """
         ms, mt = self.masks[SVG_MASK_SPATIAL], self.masks[SVG_MASK_TEMPORAL]
+        if self.layout != "explicit":
+            if self.layout == "fused":
+                svg_permute_qkv(self.geom, None, k, v, None, self.kp, self.vp, self.labels,
+                                stream=stream)
+            svg_sparse_attention_fused(self.geom, q, k, v, self.kp, self.vp, self.labels,
+                                       ms.row_ptr, ms.col_idx, mt.row_ptr, mt.col_idx, o, lse,
+                                       stream=stream)
+            return
         svg_permute_qkv(self.geom, q, k, v, self.qp, self.kp, self.vp, self.labels,
                         stream=stream)
         svg_sparse_attention(self.geom, q, k, v, self.qp, self.kp, self.vp, self.labels,
