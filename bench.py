@@ -265,12 +265,12 @@ def run_capture(args, wl):
             g, q, k, v, kp, vp, layer.labels, m[0].row_ptr, m[0].col_idx, m[1].row_ptr,
             m[1].col_idx, o)
     fns = {
-        # the attention kernel of the default (fused) layout
-        "attention": fused_attention(fu, fu.kp, fu.vp),
-        "attention_gathered": fused_attention(ga, None, None),
-        "attention_explicit": lambda: svg.svg_sparse_attention(
+        # the attention kernel of the default (explicit) layout
+        "attention": lambda: svg.svg_sparse_attention(
             g, q, k, v, ex.qp, ex.kp, ex.vp, ex.labels, ex.masks[0].row_ptr,
             ex.masks[0].col_idx, ex.masks[1].row_ptr, ex.masks[1].col_idx, o, ex.op),
+        "attention_fused": fused_attention(fu, fu.kp, fu.vp),
+        "attention_gathered": fused_attention(ga, None, None),
         "profile": lambda: fu.profile(q, k, v, rows),
         "permute": lambda: svg.svg_permute_qkv(g, q, k, v, ex.qp, ex.kp, ex.vp, ex.labels),
     }
@@ -300,7 +300,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--capture", choices=["attention", "attention_gathered", "attention_explicit",
+    ap.add_argument("--capture", choices=["attention", "attention_fused", "attention_gathered",
                                           "profile", "permute"],
                     help="small case for an ncu capture: run one kernel 3 times on the "
                          "workload with --heads heads, print per-launch ms, no JSON line")

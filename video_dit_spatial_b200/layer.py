@@ -8,12 +8,16 @@ mask; temporal outputs are moved back. This class only owns device buffers
 one stream; every step is a libsvg kernel.
 
 `layout` chooses how the layout transformation is done:
-  "explicit"  permute Q, K, V of temporal heads, attend, un-permute O;
+  "explicit"  permute Q, K, V of temporal heads, attend, un-permute O (the
+              default: the fastest);
   "fused"     permute K, V only; the attention kernel gathers the query rows of
               temporal heads in position-major order and stores each output row
-              at its frame-major place (no Q or O copies, no un-permute pass);
+              at its frame-major place (no Q or O copies, no un-permute pass;
+              about 1 % slower, since the row gathers cost about what the
+              dropped passes save);
   "gathered"  nothing is permuted: key/value rows are gathered in the kernel
-              too (least memory; row gathers are slower than tiled loads).
+              too (least memory; far slower, row gathers move fewer bytes per
+              cycle than tiled loads).
 "fused" and "gathered" need 128-row query blocks; they give the same bits as
 "explicit".
 """
@@ -49,7 +53,7 @@ class SparseVideoGenLayer:
                  layout: Optional[str] = None):
         self.geom = geom
         if layout is None:
-            layout = "fused" if geom.block_q == 128 else "explicit"
+            layout = "explicit"
         if layout not in LAYOUTS:
             raise ValueError(f"layout must be one of {LAYOUTS}")
         self.layout = layout
