@@ -5,25 +5,30 @@
 // the mean squared error of the outputs; the mask with the smaller error names
 // the head's type.
 //
-// One CTA = one (b*H + h, mask X in {spatial, temporal}, tile of 128 sampled
-// rows). It runs flash attention of its 128 gathered query rows over ALL keys
-// (128-key tiles, TMA-fed), keeping two online softmaxes side by side: the
-// full one and the token-level masked one, each with its own running maximum.
+// One CTA = one (b*H + h, tile of 128 sampled rows). It runs flash attention of
+// its 128 gathered query rows over ALL keys (64-key tiles, TMA-fed) and keeps
+// three online softmaxes side by side: the full one and the two token-level
+// masked ones, each with its own running maximum. The exponentials are taken
+// once, for the full softmax; each masked probability is the full one times
+// 2^(m_full - m_mask) on the keys its mask allows.
 //
 // 320 threads: warps 0-7 softmax, warp 8 TMA producer, warp 9 MMA issuer.
 // Warps w and w+4 own the same 32 query rows (TMEM lanes 32*(w%4)..+31) and
-// split each 128-key tile into columns [0,64) and [64,128); they exchange row
-// maxima through shared memory (one 64-thread named barrier per warp pair)
-// and keep partial row sums that are added once at the end.
-// Tensor memory: S double buffer (columns 0 and 128), O_full (256), O_X
-// (256 + d); P_full and P_X (bf16) overwrite the two halves of their S buffer.
-// The allowed keys of a row inside a tile are at most a few index runs
-// (spatial: the frames [f-s, f+s]; temporal: positions [p-w, p+w] of each
-// frame; text keys always), built as bit ranges. P_X = P_full * 2^(mF - mX) on
-// allowed keys; the masked product P_X V is skipped for key tiles where no row
-// of the CTA has an allowed key. Each CTA reduces sum((O_X - O_full)^2) over
-// its rows in a fixed order into the workspace; a second kernel adds the
-// tiles in a fixed order and labels the head.
+// split each 64-key tile into keys [0,32) and [32,64); they exchange row maxima
+// through shared memory (one 64-thread named barrier per warp pair) and keep
+// partial row sums that are added once at the end.
+// Tensor memory: S double buffer (64 columns each at 0 and 64), O_full (128),
+// O_spatial (128 + d), O_temporal (128 + 2d). P_full and P_temporal (bf16)
+// overwrite the two halves of their S buffer and feed their PV products from
+// tensor memory; P_spatial goes to a double-buffered swizzled tile in shared
+// memory and feeds its product from there. A masked product is skipped for key
+// tiles where no row of the CTA has an allowed key, and a warp rewrites its
+// rows of a P_spatial buffer only when they are not already zero. The allowed keys of a row
+// inside a tile are at most a few index runs (spatial: the frames [f-s, f+s];
+// temporal: positions [p-w, p+w] of each frame; text keys always), built as
+// bit ranges. Each CTA reduces sum((O_X - O_full)^2) over its rows in a fixed
+// order into the workspace; a second kernel adds the tiles in a fixed order
+// and labels the head.
 #include <mutex>
 
 #include "internal.h"
@@ -36,42 +41,47 @@ constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr int kProducerWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kTile = 128;  // sampled rows per CTA and keys per tile
-constexpr int kHalf = 64;   // keys per softmax thread per tile
+constexpr int kRows = 128;  // sampled rows per CTA
+constexpr int kKeys = 64;   // keys per tile
+constexpr int kHalf = 32;   // keys per softmax thread per tile
+constexpr int kKStages = 4;
+constexpr int kVStages = 3;
 constexpr float kRebaseLog2 = 8.0f;
 
 struct PBarriers {
-  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_full, o_final, drain;
   uint32_t tmem_base;
   int abort_flag;
-  int x_active[2][kSoftmaxWarps];
-  float xmax[2][2][128];  // [half][full, masked][row]
-  float xsum[2][2][128];  // [half][full, masked][row]
-  float red[2][128];
+  int x_active[2][2][kSoftmaxWarps];  // [buffer][mask][warp]
+  float xmax[2][3][kRows];            // [half][full, spatial, temporal][row]
+  float xsum[2][3][kRows];            // [half][full, spatial, temporal][row]
+  float red[2][2][kRows];             // [half][spatial, temporal][row]
   int pair_fail[4][2];
 };
 
 template <int D>
 struct PCfg {
   static constexpr int kPanels = D / 64;
-  static constexpr int kPanel = 128 * 128;  // 128 rows x 128 B
-  static constexpr int kQBytes = kPanels * kPanel;
-  static constexpr int kKVBytes = kPanels * kPanel;
-  // K is released right after its QK product, V only after its PV products,
-  // so K gets the deeper ring.
-  static constexpr int kKStages = 3;
-  static constexpr int kVStages = D == 128 ? 2 : 3;
+  static constexpr int kQPanel = kRows * 128;   // 128 rows x 128 B
+  static constexpr int kKVPanel = kKeys * 128;  // 64 rows x 128 B
+  static constexpr int kQBytes = kPanels * kQPanel;
+  static constexpr int kKVBytes = kPanels * kKVPanel;
+  static constexpr int kPBytes = kRows * kKeys * 2;  // one masked P tile, K-major swizzled
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kKStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kVStages * kKVBytes;
+  static constexpr int kOffP = kOffV + kVStages * kKVBytes;  // P_spatial [buffer]
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
   static constexpr int kBarBytes = (static_cast<int>(sizeof(PBarriers)) + 127) / 128 * 128;
   static constexpr int kUsed = kOffBar + kBarBytes + 1024;
   static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColOF = 256, kColOX = 256 + D;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 64;
+  static constexpr uint32_t kColOF = 128, kColOS = 128 + D, kColOT = 128 + 2 * D;
+  static_assert(kColOT + D <= kTmemCols, "accumulators must fit tensor memory");
+  static_assert(kOffP % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
   static_assert(kOffBar + kBarBytes + 1024 <= kSmem, "bookkeeping must fit the allocation");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
@@ -99,6 +109,52 @@ __device__ __forceinline__ void softmax_sync() {
   asm volatile("bar.sync 5, 256;" ::: "memory");
 }
 
+// Bits [a, b) of a 32-bit word, for 0 <= a, b <= 32 (empty when b <= a).
+__device__ __forceinline__ uint32_t bit_range32(int a, int b) {
+  a = max(a, 0);
+  b = min(b, 32);
+  if (b <= a) return 0u;
+  return static_cast<uint32_t>((1ull << b) - (1ull << a));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Masked probabilities of one half tile for one mask, from the full ones.
+//   SHAPE 0: some keys allowed (per-key selection), 1: no key allowed in the
+//   warp, 2: every key allowed in the warp, 3: the masked base is far below the
+//   full one for some row, so allowed keys take their own exponential.
+template <int SHAPE>
+__device__ __forceinline__ void masked_pass(const float (&f)[kHalf], const uint32_t (&sr)[kHalf],
+                                            uint32_t bits, float k, bool direct, float scale_log2,
+                                            float u, uint32_t (&pk)[kHalf / 2], float& sum) {
+  float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kHalf / 2; ++i) {
+    float g0, g1;
+    if (SHAPE == 1) {
+      g0 = g1 = 0.0f;
+    } else {
+      ffma2(g0, g1, f[2 * i], f[2 * i + 1], k, k, 0.0f, 0.0f);
+      if (SHAPE == 3 && direct) {
+        g0 = fast_exp2(fmaf(u2f(sr[2 * i]), scale_log2, -u));
+        g1 = fast_exp2(fmaf(u2f(sr[2 * i + 1]), scale_log2, -u));
+      }
+      if (SHAPE != 2) {
+        g0 = (bits >> (2 * i)) & 1u ? g0 : 0.0f;
+        g1 = (bits >> (2 * i + 1)) & 1u ? g1 : 0.0f;
+      }
+      fadd2(s0, s1, s0, s1, g0, g1);
+    }
+    pk[i] = pack_bf16x2(g0, g1);
+  }
+  sum = s0 + s1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_constant__ ProfParams p) {
   using C = PCfg<D>;
@@ -108,16 +164,14 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
+  uint8_t* sP = smem + C::kOffP;
   PBarriers* bar = reinterpret_cast<PBarriers*>(smem + C::kOffBar);
   volatile int* abort_flag = &bar->abort_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  // Launch order: every temporal-mask CTA (the slower kind: its allowed keys
-  // reach every frame) before any spatial-mask CTA, heads in order.
   const int tile = blockIdx.x;
   const int bh = blockIdx.y;
-  const int X = 1 - static_cast<int>(blockIdx.z);  // 0: spatial mask, 1: temporal mask
   const int n = p.nkt;
 
   if (warp == 0) {
@@ -126,9 +180,11 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     tc_fence_before();
   }
   if (tid == 32) {
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
     }
@@ -149,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
   const int half = (tid >> 7) & 1;
   int qrow = -1;
   if (warp < kSoftmaxWarps) {
-    const int si = tile * kTile + row;
+    const int si = tile * kRows + row;
     if (si < p.n_samples) {
       const int r = __ldg(p.sample_idx + si);
       if (r >= 0 && r < p.Nv) {
@@ -165,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       const int c = half * (D / 16) + cc;
       const uint4 v = qrow >= 0 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
       const int pn = c >> 3, ci = c & 7;
-      *reinterpret_cast<uint4*>(sQ + pn * C::kPanel + row * 128 + ((ci ^ (row & 7)) << 4)) = v;
+      *reinterpret_cast<uint4*>(sQ + pn * C::kQPanel + row * 128 + ((ci ^ (row & 7)) << 4)) = v;
     }
     fence_proxy_async_smem();
   }
@@ -182,38 +238,38 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       bool ok = true;
       for (int j = 0; ok && j <= n; ++j) {
         if (j < n) {
-          const int st = j % C::kKStages;
-          ok = mbar_wait(&bar->k_empty[st], ((j / C::kKStages) & 1) ^ 1, abort_flag, p.status);
+          const int st = j % kKStages;
+          ok = mbar_wait(&bar->k_empty[st], ((j / kKStages) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
           mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kPanel, &p.tm_k, &bar->k_full[st],
-                             pn * 64, j * kTile, bh, keep);
+            tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kKVPanel, &p.tm_k, &bar->k_full[st],
+                             pn * 64, j * kKeys, bh, keep);
           k_issued = j + 1;
         }
         if (j >= 1) {
           const int jv = j - 1;
-          const int st = jv % C::kVStages;
-          ok = mbar_wait(&bar->v_empty[st], ((jv / C::kVStages) & 1) ^ 1, abort_flag, p.status);
+          const int st = jv % kVStages;
+          ok = mbar_wait(&bar->v_empty[st], ((jv / kVStages) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
           mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kPanel, &p.tm_v, &bar->v_full[st],
-                             pn * 64, jv * kTile, bh, keep);
+            tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kKVPanel, &p.tm_v, &bar->v_full[st],
+                             pn * 64, jv * kKeys, bh, keep);
           v_issued = jv + 1;
         }
       }
       if (*abort_flag) {
         // Let every copy this thread started land before the CTA retires.
-        for (int j = (k_issued > C::kKStages ? k_issued - C::kKStages : 0); j < k_issued; ++j) {
+        for (int j = (k_issued > kKStages ? k_issued - kKStages : 0); j < k_issued; ++j) {
           long long t0 = clock64();
-          while (!mbar_try_wait(&bar->k_full[j % C::kKStages], (j / C::kKStages) & 1) &&
+          while (!mbar_try_wait(&bar->k_full[j % kKStages], (j / kKStages) & 1) &&
                  clock64() - t0 < kWaitLimitCycles) {
           }
         }
-        for (int j = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); j < v_issued; ++j) {
+        for (int j = (v_issued > kVStages ? v_issued - kVStages : 0); j < v_issued; ++j) {
           long long t0 = clock64();
-          while (!mbar_try_wait(&bar->v_full[j % C::kVStages], (j / C::kVStages) & 1) &&
+          while (!mbar_try_wait(&bar->v_full[j % kVStages], (j / kVStages) & 1) &&
                  clock64() - t0 < kWaitLimitCycles) {
           }
         }
@@ -221,56 +277,67 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     }
   } else if (warp == kMmaWarp) {
     if (lane_id() == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTile, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kKeys, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
-      bool x_started = false;
+      const uint32_t p_addr = smem_u32(sP);
+      bool started[2] = {false, false};
       for (int j = 0; j <= n; ++j) {
         if (j < n) {
-          const int st = j % C::kKStages;
+          const int st = j % kKStages;
           const uint32_t s_col = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
-          if (!mbar_wait(&bar->k_full[st], (j / C::kKStages) & 1, abort_flag, p.status)) break;
+          if (!mbar_wait(&bar->k_full[st], (j / kKStages) & 1, abort_flag, p.status)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kPanel + (kk & 3) * 32;
-            mma_bf16_ss(s_col, sdesc_sw128(q_addr + off, 16, 1024),
-                        sdesc_sw128(k_addr + st * C::kKVBytes + off, 16, 1024), idesc_qk,
-                        kk > 0 ? 1u : 0u);
+            const uint32_t off = (kk & 3) * 32;
+            mma_bf16_ss(s_col, sdesc_sw128(q_addr + (kk >> 2) * C::kQPanel + off, 16, 1024),
+                        sdesc_sw128(k_addr + st * C::kKVBytes + (kk >> 2) * C::kKVPanel + off, 16,
+                                    1024),
+                        idesc_qk, kk > 0 ? 1u : 0u);
           }
           tc_commit(&bar->s_full[j & 1]);
           tc_commit(&bar->k_empty[st]);  // K(j) is free once QK_j retires
         }
         if (j >= 1) {
           const int jj = j - 1;
-          const int st = jj % C::kVStages;
+          const int st = jj % kVStages;
           const int sb = jj & 1;
-          const uint32_t p_col = tmem + (sb ? C::kColS1 : C::kColS0);
+          const uint32_t pf_col = tmem + (sb ? C::kColS1 : C::kColS0);
           if (!mbar_wait(&bar->p_full[sb], (jj >> 1) & 1, abort_flag, p.status)) break;
-          if (!mbar_wait(&bar->v_full[st], (jj / C::kVStages) & 1, abort_flag, p.status)) break;
+          if (!mbar_wait(&bar->v_full[st], (jj / kVStages) & 1, abort_flag, p.status)) break;
           tc_fence_after();
-          const volatile int* xa = bar->x_active[sb];
-          int x_any = 0;
+          int active[2] = {0, 0};
 #pragma unroll
-          for (int w = 0; w < kSoftmaxWarps; ++w) x_any |= xa[w];
+          for (int m = 0; m < 2; ++m) {
+            const volatile int* xa = bar->x_active[sb][m];
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t b = sdesc_sw128(v_addr + st * C::kKVBytes + kk * 16 * 128, C::kPanel,
-                                           1024);
-            mma_bf16_ts(tmem + C::kColOF, p_col + kk * 8, b, idesc_pv,
-                        (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int w = 0; w < kSoftmaxWarps; ++w) active[m] |= xa[w];
           }
-          if (x_any) {
+          const uint32_t vb = v_addr + st * C::kKVBytes;
 #pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
-              const uint64_t b = sdesc_sw128(v_addr + st * C::kKVBytes + kk * 16 * 128,
-                                             C::kPanel, 1024);
-              mma_bf16_ts(tmem + C::kColOX, p_col + 64 + kk * 8, b, idesc_pv,
-                          (x_started || kk > 0) ? 1u : 0u);
-            }
-            x_started = true;
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            mma_bf16_ts(tmem + C::kColOF, pf_col + kk * 8,
+                        sdesc_sw128(vb + kk * 16 * 128, C::kKVPanel, 1024), idesc_pv,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
+          if (active[0]) {  // spatial: P from shared memory
+            const uint32_t pm = p_addr + sb * C::kPBytes;
+#pragma unroll
+            for (int kk = 0; kk < kKeys / 16; ++kk)
+              mma_bf16_ss(tmem + C::kColOS, sdesc_sw128(pm + kk * 32, 16, 1024),
+                          sdesc_sw128(vb + kk * 16 * 128, C::kKVPanel, 1024), idesc_pv,
+                          (started[0] || kk > 0) ? 1u : 0u);
+            started[0] = true;
+          }
+          if (active[1]) {  // temporal: P from the upper half of the S buffer
+#pragma unroll
+            for (int kk = 0; kk < kKeys / 16; ++kk)
+              mma_bf16_ts(tmem + C::kColOT, pf_col + kKeys / 2 + kk * 8,
+                          sdesc_sw128(vb + kk * 16 * 128, C::kKVPanel, 1024), idesc_pv,
+                          (started[1] || kk > 0) ? 1u : 0u);
+            started[1] = true;
           }
           tc_commit(&bar->v_empty[st]);
           tc_commit(&bar->o_full);
@@ -286,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int group = warp & 3;  // rows 32*group .. +31 (TMEM lane quarter)
+    const int group = warp & 3;       // rows 32*group .. +31 (TMEM lane quarter)
     const int c_base = half * kHalf;  // this thread's key columns within a tile
     const bool row_valid = qrow >= 0;
     const int qi = row_valid ? qrow : 0;
@@ -295,52 +362,54 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     // Allowed video keys of this row: spatial = the frames [f_i - s, f_i + s]
     // (one index run); temporal = positions [p_i - w, p_i + w] of every frame
     // (one run per frame). Text keys [Nv, N) are allowed by both.
-    const int s_lo = max(f_i - p.s, 0) * p.P;  // frames [f_i - s, f_i + s] as one index run
+    const int s_lo = max(f_i - p.s, 0) * p.P;
     const int s_hi = static_cast<int>(min(static_cast<long long>(f_i) + p.s + 1,
                                           static_cast<long long>(p.T))) * p.P;
     const int t_lo = max(p_i - p.w, 0);
     const int t_hi = static_cast<int>(
         min(static_cast<long long>(p_i) + p.w, static_cast<long long>(p.P - 1)));
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(group * 32) << 16);
-    float mF = -INFINITY, lF = 0.0f, mX = -INFINITY, lX = 0.0f;
+    const uint32_t p_row = smem_u32(sP) + row * 128;
+    // running bases (log2 units) and sums of the full, spatial, temporal softmax
+    float m[3] = {-INFINITY, -INFINITY, -INFINITY};
+    float l[3] = {0.0f, 0.0f, 0.0f};
     bool ok = true;
     int fs0 = 0;  // start of the frame holding this thread's first key of the tile
+    bool ps_zero[2] = {false, false};  // this warp's rows of P_spatial[buffer] hold zeros
     for (int j = 0; j < n; ++j) {
       const int sb = j & 1;
       const uint32_t s_col = lane_base + (sb ? C::kColS1 : C::kColS0);
-      const int k0 = j * kTile + c_base;       // first key of this thread's half
+      const int k0 = j * kKeys + c_base;  // first key of this thread's half
       const int kvalid = max(0, min(kHalf, p.N - k0));
-      const int k_end = k0 + kvalid;           // exclusive
-      uint32_t bits[2] = {0u, 0u};  // allowed keys k0 + [0, 64) of this row
+      const int k_end = k0 + kvalid;  // exclusive
+      uint32_t bits[2] = {0u, 0u};    // allowed keys k0 + [0, 32): spatial, temporal
       if (row_valid && kvalid > 0) {
-        if (k_end > p.Nv) set_bit_range64(bits, max(p.Nv, k0) - k0, kvalid);
+        if (k_end > p.Nv) {
+          const uint32_t text = bit_range32(max(p.Nv, k0) - k0, kvalid);
+          bits[0] = bits[1] = text;
+        }
         if (k0 < p.Nv) {
           const int v_end = min(k_end, p.Nv);
-          if (X == 0) {
-            set_bit_range64(bits, max(s_lo, k0) - k0, min(s_hi, v_end) - k0);
-          } else {
-            // frames overlapping the half tile (at most two when P >= 64);
-            // fs0 tracks the start of the frame holding k0 across tiles
-            while (fs0 + p.P <= k0) fs0 += p.P;
-            for (int fs = fs0; fs < v_end; fs += p.P)
-              set_bit_range64(bits, max(fs + t_lo, k0) - k0, min(fs + t_hi + 1, v_end) - k0);
-          }
+          bits[0] |= bit_range32(max(s_lo, k0) - k0, min(s_hi, v_end) - k0);
+          // frames overlapping the half tile; fs0 tracks the start of the frame
+          // holding k0 across tiles
+          while (fs0 + p.P <= k0) fs0 += p.P;
+          for (int fs = fs0; fs < v_end; fs += p.P)
+            bits[1] |= bit_range32(fs + t_lo - k0, min(fs + t_hi + 1, v_end) - k0);
         }
       }
-      const bool any_x = (bits[0] | bits[1]) != 0u;
-      const int warp_any = __any_sync(0xffffffffu, any_x) ? 1 : 0;
 
       if (ok && !mbar_wait(&bar->s_full[sb], (j >> 1) & 1, abort_flag, p.status)) ok = false;
       // Both warps of a pair must take the same path through pair_sync (an
       // unbounded barrier), so they agree on leaving the loop through it.
       if (__any_sync(0xffffffffu, !ok)) ok = false;
       if (lane_id() == 0) bar->pair_fail[group][half] = ok ? 0 : 1;
-      float a0 = -INFINITY, a1 = -INFINITY, b0 = -INFINITY, b1 = -INFINITY;
+      float a0 = -INFINITY, a1 = -INFINITY;
+      float bmax[2] = {-INFINITY, -INFINITY};
       uint32_t sr[kHalf];
       if (ok) {
         tc_fence_after();
-        tmem_ld_32x32b_x32(s_col + c_base, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld_32x32b_x32(s_col + c_base + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld_32x32b_x32(s_col + c_base, sr);
         tmem_ld_wait();
         reg_fence(sr);
         if (kvalid < kHalf) {  // only the last tile is ragged
@@ -353,28 +422,33 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
           a0 = fmax3(a0, u2f(sr[c]), u2f(sr[c + 1]));
           a1 = fmax3(a1, u2f(sr[c + 2]), u2f(sr[c + 3]));
         }
-        // The masked maximum of this half can only move the masked base when
-        // the half's full maximum exceeds mX + 2^8; otherwise report -inf: the
-        // combined decision and the new base are unchanged.
-        const bool need_m = any_x && fmaxf(a0, a1) * p.scale_log2 > mX + kRebaseLog2;
-        if (__any_sync(0xffffffffu, need_m)) {
+        // A masked maximum of this half can only move its masked base when the
+        // half's full maximum exceeds that base + 2^8; otherwise report -inf:
+        // the combined decision and the new base are unchanged.
+        const float hmax = fmaxf(a0, a1) * p.scale_log2;
 #pragma unroll
-          for (int c = 0; c < kHalf; c += 4) {
-            const float x0 = ((bits[c >> 5] >> (c & 31)) & 1u) ? u2f(sr[c]) : -INFINITY;
-            const float x1 = ((bits[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) ? u2f(sr[c + 1]) : -INFINITY;
-            const float x2 = ((bits[(c + 2) >> 5] >> ((c + 2) & 31)) & 1u) ? u2f(sr[c + 2]) : -INFINITY;
-            const float x3 = ((bits[(c + 3) >> 5] >> ((c + 3) & 31)) & 1u) ? u2f(sr[c + 3]) : -INFINITY;
-            b0 = fmax3(b0, x0, x1);
-            b1 = fmax3(b1, x2, x3);
+        for (int x = 0; x < 2; ++x) {
+          const bool need = bits[x] != 0u && hmax > m[1 + x] + kRebaseLog2;
+          if (__any_sync(0xffffffffu, need)) {
+            float b0 = -INFINITY, b1 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kHalf; c += 2) {
+              b0 = fmaxf(b0, (bits[x] >> c) & 1u ? u2f(sr[c]) : -INFINITY);
+              b1 = fmaxf(b1, (bits[x] >> (c + 1)) & 1u ? u2f(sr[c + 1]) : -INFINITY);
+            }
+            bmax[x] = fmaxf(b0, b1);
           }
         }
       }
       // exchange the half-row maxima with the partner warp
       bar->xmax[half][0][row] = fmaxf(a0, a1);
-      bar->xmax[half][1][row] = fmaxf(b0, b1);
+      bar->xmax[half][1][row] = bmax[0];
+      bar->xmax[half][2][row] = bmax[1];
       pair_sync(group);
-      const float tF = fmaxf(bar->xmax[0][0][row], bar->xmax[1][0][row]) * p.scale_log2;
-      const float tX = fmaxf(bar->xmax[0][1][row], bar->xmax[1][1][row]) * p.scale_log2;
+      float t[3];
+#pragma unroll
+      for (int x = 0; x < 3; ++x)
+        t[x] = fmaxf(bar->xmax[0][x][row], bar->xmax[1][x][row]) * p.scale_log2;
       const int pair_failed = bar->pair_fail[group][0] | bar->pair_fail[group][1];
       pair_sync(group);  // the exchange slots are rewritten next tile
       if (pair_failed) {
@@ -382,111 +456,97 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
         break;
       }
 
-      const bool rbF = tF > mF + kRebaseLog2;
-      const bool rbX = tX > mX + kRebaseLog2;
-      const float mF_new = rbF ? tF : mF, mX_new = rbX ? tX : mX;
-      const float aF = rbF ? fast_exp2(mF - mF_new) : 1.0f;
-      const float aX = rbX ? fast_exp2(mX - mX_new) : 1.0f;
-      const float uF = mF_new == -INFINITY ? 0.0f : mF_new;
-      const float uX = mX_new == -INFINITY ? 0.0f : mX_new;
-      // P_X = P_full * 2^(mF - mX) on allowed keys, unless the masked base is
-      // so far below the full one that 2^(x - mF) could flush to zero; those
-      // (rare) warps evaluate the masked exponentials directly.
-      // (With no allowed key seen yet, mX is -inf and every P_X is zero.)
-      const float gap = uF - uX;
-      const bool direct = mX_new != -INFINITY && gap > 64.0f;
-      const float kX = direct ? 0.0f : fast_exp2(gap);
-      const bool warp_direct = __any_sync(0xffffffffu, direct);
-      // Warp-uniform shapes of the allowed-key set of this half tile.
-      const bool w_none = __all_sync(0xffffffffu, (bits[0] | bits[1]) == 0u);
-      const bool w_all = __all_sync(0xffffffffu, (bits[0] & bits[1]) == 0xffffffffu);
-      const int shape = warp_direct ? 3 : (w_none ? 1 : (w_all ? 2 : 0));
-      float sF0 = 0.0f, sF1 = 0.0f, sX0 = 0.0f, sX1 = 0.0f;
+      bool rb[3];
+      float m_new[3], alpha[3], u[3];
 #pragma unroll
-      for (int ch = 0; ch < kHalf / 32; ++ch) {
-        uint32_t pkF[16], pkX[16];
-        if (shape == 1) {  // no allowed key in this half for the whole warp
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c0 = ch * 32 + 2 * i;
-            float y0, y1;
-            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
-            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
-            fadd2(sF0, sF1, sF0, sF1, f0, f1);
-            pkF[i] = pack_bf16x2(f0, f1);
-            pkX[i] = 0u;
-          }
-        } else if (shape == 2) {  // every key allowed for the whole warp
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c0 = ch * 32 + 2 * i;
-            float y0, y1, g0, g1;
-            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
-            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
-            ffma2(g0, g1, f0, f1, kX, kX, 0.0f, 0.0f);
-            fadd2(sF0, sF1, sF0, sF1, f0, f1);
-            fadd2(sX0, sX1, sX0, sX1, g0, g1);
-            pkF[i] = pack_bf16x2(f0, f1);
-            pkX[i] = pack_bf16x2(g0, g1);
-          }
-        } else if (shape == 0) {  // general: per-key selection
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c0 = ch * 32 + 2 * i;
-            float y0, y1;
-            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
-            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
-            const float g0 = ((bits[ch] >> (2 * i)) & 1u) ? f0 * kX : 0.0f;
-            const float g1 = ((bits[ch] >> (2 * i + 1)) & 1u) ? f1 * kX : 0.0f;
-            fadd2(sF0, sF1, sF0, sF1, f0, f1);
-            fadd2(sX0, sX1, sX0, sX1, g0, g1);
-            pkF[i] = pack_bf16x2(f0, f1);
-            pkX[i] = pack_bf16x2(g0, g1);
-          }
-        } else {  // some row's masked base is far below its full base
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c0 = ch * 32 + 2 * i;
-            float y0, y1;
-            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -uF, -uF);
-            const float f0 = fast_exp2(y0), f1 = fast_exp2(y1);
-            const bool in0 = (bits[ch] >> (2 * i)) & 1u;
-            const bool in1 = (bits[ch] >> (2 * i + 1)) & 1u;
-            float g0 = in0 ? f0 * kX : 0.0f;
-            float g1 = in1 ? f1 * kX : 0.0f;
-            if (direct) {
-              g0 = in0 ? fast_exp2(fmaf(u2f(sr[c0]), p.scale_log2, -uX)) : 0.0f;
-              g1 = in1 ? fast_exp2(fmaf(u2f(sr[c0 + 1]), p.scale_log2, -uX)) : 0.0f;
-            }
-            fadd2(sF0, sF1, sF0, sF1, f0, f1);
-            fadd2(sX0, sX1, sX0, sX1, g0, g1);
-            pkF[i] = pack_bf16x2(f0, f1);
-            pkX[i] = pack_bf16x2(g0, g1);
-          }
-        }
-        // keys k -> column k/2: this half's 64 keys fill 32 columns
-        tmem_st_32x32b_x16(s_col + half * 32 + ch * 16, pkF);
-        tmem_st_32x32b_x16(s_col + 64 + half * 32 + ch * 16, pkX);
+      for (int x = 0; x < 3; ++x) {
+        rb[x] = t[x] > m[x] + kRebaseLog2;
+        m_new[x] = rb[x] ? t[x] : m[x];
+        alpha[x] = rb[x] ? fast_exp2(m[x] - m_new[x]) : 1.0f;  // exp2(-inf) = 0
+        u[x] = m_new[x] == -INFINITY ? 0.0f : m_new[x];
       }
-      lF = lF * aF + (sF0 + sF1);
-      lX = lX * aX + (sX0 + sX1);
-      mF = mF_new;
-      mX = mX_new;
+      // full probabilities of this half tile
+      float f[kHalf];
+      uint32_t pkF[kHalf / 2];
+      float sF0 = 0.0f, sF1 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < kHalf / 2; ++i) {
+        float y0, y1;
+        ffma2(y0, y1, u2f(sr[2 * i]), u2f(sr[2 * i + 1]), p.scale_log2, p.scale_log2, -u[0],
+              -u[0]);
+        f[2 * i] = fast_exp2(y0);
+        f[2 * i + 1] = fast_exp2(y1);
+        fadd2(sF0, sF1, sF0, sF1, f[2 * i], f[2 * i + 1]);
+        pkF[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+      }
+      tmem_st_32x32b_x16(s_col + half * (kHalf / 2), pkF);
+      float sum[3] = {sF0 + sF1, 0.0f, 0.0f};
+      // masked probabilities: P_X = P_full * 2^(u_full - u_X) on allowed keys,
+      // unless the masked base is so far below the full one that the full
+      // probabilities could flush to zero; those rows (rare) take the masked
+      // exponentials directly. (With no allowed key seen yet, m_X is -inf and
+      // every P_X is zero.)
+      int warp_any[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const float gap = u[0] - u[1 + x];
+        const bool direct = m_new[1 + x] != -INFINITY && gap > 64.0f;
+        const float kx = direct ? 0.0f : fast_exp2(gap);
+        const bool w_none = __all_sync(0xffffffffu, bits[x] == 0u);
+        const bool w_all = __all_sync(0xffffffffu, bits[x] == 0xffffffffu);
+        const bool w_direct = __any_sync(0xffffffffu, direct);
+        warp_any[x] = w_none ? 0 : 1;
+        uint32_t pk[kHalf / 2];
+        if (w_direct)
+          masked_pass<3>(f, sr, bits[x], kx, direct, p.scale_log2, u[1 + x], pk, sum[1 + x]);
+        else if (w_none)
+          masked_pass<1>(f, sr, bits[x], kx, direct, p.scale_log2, u[1 + x], pk, sum[1 + x]);
+        else if (w_all)
+          masked_pass<2>(f, sr, bits[x], kx, direct, p.scale_log2, u[1 + x], pk, sum[1 + x]);
+        else
+          masked_pass<0>(f, sr, bits[x], kx, direct, p.scale_log2, u[1 + x], pk, sum[1 + x]);
+        if (x == 1) {
+          // temporal: keys k -> column 32 + k/2 of the S buffer (its upper half)
+          tmem_st_32x32b_x16(s_col + kKeys / 2 + half * (kHalf / 2), pk);
+        } else if (!(w_none && ps_zero[sb])) {
+          // spatial: this row's 32 keys = chunks 4*half .. 4*half+3 of its
+          // 128-byte row in the shared-memory tile
+          const uint32_t base = p_row + sb * C::kPBytes;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int chunk = 4 * half + c;
+            st_shared_v4(base + ((chunk ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1],
+                         pk[4 * c + 2], pk[4 * c + 3]);
+          }
+          ps_zero[sb] = w_none;
+        }
+      }
+      fence_proxy_async_smem();
+#pragma unroll
+      for (int x = 0; x < 3; ++x) {
+        l[x] = l[x] * alpha[x] + sum[x];
+        m[x] = m_new[x];
+      }
       tmem_st_wait();
-      if (lane_id() == 0) bar->x_active[sb][warp] = warp_any;
+      if (lane_id() == 0) {
+        bar->x_active[sb][0][warp] = warp_any[0];
+        bar->x_active[sb][1][warp] = warp_any[1];
+      }
 
-      // Re-base this half's columns of O_full / O_X once PV_{j-1} has landed.
-      const bool wF = __any_sync(0xffffffffu, rbF);
-      const bool wX = __any_sync(0xffffffffu, rbX);
-      if (j > 0 && (wF || wX)) {
+      // Re-base this half's columns of the moved accumulators once PV_{j-1}
+      // has landed.
+      bool wrb[3];
+#pragma unroll
+      for (int x = 0; x < 3; ++x) wrb[x] = __any_sync(0xffffffffu, rb[x]);
+      if (j > 0 && (wrb[0] || wrb[1] || wrb[2])) {
         // A failed wait is reported through the pair exchange of the next tile.
         if (!mbar_wait(&bar->o_full, (j - 1) & 1, abort_flag, p.status)) ok = false;
         tc_fence_after();
 #pragma unroll
-        for (int which = 0; which < 2 && ok; ++which) {
-          if (which == 0 ? !wF : !wX) continue;
-          const float a = which == 0 ? aF : aX;
-          const uint32_t ocol = lane_base + (which == 0 ? C::kColOF : C::kColOX) + half * (D / 2);
+        for (int x = 0; x < 3 && ok; ++x) {
+          if (!wrb[x]) continue;
+          const uint32_t ocol =
+              lane_base + (x == 0 ? C::kColOF : (x == 1 ? C::kColOS : C::kColOT)) + half * (D / 2);
 #pragma unroll
           for (int ch = 0; ch < D / 64; ++ch) {
             uint32_t o[32];
@@ -494,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
             tmem_ld_wait();
             reg_fence(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * a);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * alpha[x]);
             tmem_st_32x32b_x32(ocol + ch * 32, o);
           }
         }
@@ -504,41 +564,52 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       mbar_arrive(&bar->p_full[sb]);
     }
 
-    // ---- per-row squared error over this half's d/2 channels
-    bar->xsum[half][0][row] = lF;
-    bar->xsum[half][1][row] = lX;
+    // ---- per-row squared errors over this half's d/2 channels
+#pragma unroll
+    for (int x = 0; x < 3; ++x) bar->xsum[half][x][row] = l[x];
     if (ok && n > 0) ok = mbar_wait(&bar->o_final, 0, abort_flag, p.status);
     softmax_sync();
-    const float LF = bar->xsum[0][0][row] + bar->xsum[1][0][row];
-    const float LX = bar->xsum[0][1][row] + bar->xsum[1][1][row];
+    float inv[3];
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      const float L = bar->xsum[0][x][row] + bar->xsum[1][x][row];
+      inv[x] = L > 0.0f ? 1.0f / L : 0.0f;
+    }
     tc_fence_after();
-    float err = 0.0f;
+    float err[2] = {0.0f, 0.0f};
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (all_ok && n > 0) {
-      const float iF = LF > 0.0f ? 1.0f / LF : 0.0f;
-      const float iX = LX > 0.0f ? 1.0f / LX : 0.0f;
 #pragma unroll
       for (int ch = 0; ch < D / 64; ++ch) {
         uint32_t oF[32], oX[32];
         tmem_ld_32x32b_x32(lane_base + C::kColOF + half * (D / 2) + ch * 32, oF);
-        tmem_ld_32x32b_x32(lane_base + C::kColOX + half * (D / 2) + ch * 32, oX);
         tmem_ld_wait();
         reg_fence(oF);
-        reg_fence(oX);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float dlt = u2f(oX[i]) * iX - u2f(oF[i]) * iF;
-          err = fmaf(dlt, dlt, err);
+        for (int x = 0; x < 2; ++x) {
+          tmem_ld_32x32b_x32(lane_base + (x == 0 ? C::kColOS : C::kColOT) + half * (D / 2) +
+                                 ch * 32,
+                             oX);
+          tmem_ld_wait();
+          reg_fence(oX);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float ox = inv[1 + x] > 0.0f ? u2f(oX[i]) * inv[1 + x] : 0.0f;
+            const float dlt = ox - u2f(oF[i]) * inv[0];
+            err[x] = fmaf(dlt, dlt, err[x]);
+          }
         }
       }
     }
-    bar->red[half][row] = row_valid ? err : 0.0f;
+    bar->red[half][0][row] = row_valid ? err[0] : 0.0f;
+    bar->red[half][1][row] = row_valid ? err[1] : 0.0f;
     if (!all_ok) atomicOr(&bar->abort_flag, 1);
     softmax_sync();
-    if (tid == 0) {
+    if (tid < 2) {
+      const int x = tid;
       float acc = 0.0f;
-      for (int i = 0; i < 128; ++i) acc += bar->red[0][i] + bar->red[1][i];
-      p.partial[(static_cast<size_t>(bh) * 2 + X) * p.n_tiles + tile] =
+      for (int i = 0; i < kRows; ++i) acc += bar->red[0][x][i] + bar->red[1][x][i];
+      p.partial[(static_cast<size_t>(bh) * 2 + x) * p.n_tiles + tile] =
           *abort_flag ? __int_as_float(0x7fc00000) : acc;
     }
   }
@@ -578,7 +649,7 @@ cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, flo
   auto kern = profile_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(pp.n_tiles, d.BH, 2), kThreads, C::kSmem, stream>>>(pp);
+  kern<<<dim3(pp.n_tiles, d.BH), kThreads, C::kSmem, stream>>>(pp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float inv = 1.0f / (static_cast<float>(pp.n_samples) * static_cast<float>(D));
@@ -589,7 +660,7 @@ cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, flo
 
 }  // namespace
 
-int32_t profile_tiles(int32_t n_samples) { return (n_samples + kTile - 1) / kTile; }
+int32_t profile_tiles(int32_t n_samples) { return (n_samples + kRows - 1) / kRows; }
 
 // ---------------------------------------------------------------------------
 // Fixed scratch for svg_profile_heads_noalloc: the per-tile partial sums live
@@ -640,8 +711,8 @@ cudaError_t launch_profile_noalloc(const Dims& d, const ProfileArgs& a, int* sta
 cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cudaStream_t stream) {
   ProfParams pp;
   memset(&pp, 0, sizeof(pp));
-  if (!make_tmap_bf16(&pp.tm_k, a.k, d.d, d.N, d.BH, kTile) ||
-      !make_tmap_bf16(&pp.tm_v, a.v, d.d, d.N, d.BH, kTile))
+  if (!make_tmap_bf16(&pp.tm_k, a.k, d.d, d.N, d.BH, kKeys) ||
+      !make_tmap_bf16(&pp.tm_v, a.v, d.d, d.N, d.BH, kKeys))
     return cudaErrorInvalidValue;
   pp.q = a.q;
   pp.sample_idx = a.sample_idx;
@@ -655,7 +726,7 @@ cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cud
   pp.P = d.P;
   pp.s = d.s;
   pp.w = d.w;
-  pp.nkt = (d.N + kTile - 1) / kTile;
+  pp.nkt = (d.N + kKeys - 1) / kKeys;
   pp.scale_log2 = d.scale * 1.4426950408889634f;
   if (d.d == 128) return launch_impl<128>(d, pp, a.labels, a.mse, stream);
   return launch_impl<64>(d, pp, a.labels, a.mse, stream);
