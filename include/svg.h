@@ -107,7 +107,11 @@ svg_status svg_build_block_mask(const svg_geom* geom, int32_t kind, int32_t* row
 
 /* ---------------------------------------------------------------------------
  * svg_profile_workspace_bytes -- host only: device workspace svg_profile_heads
- * needs for n_samples sampled rows (partial sums of the MSE reduction).
+ * needs for n_samples sampled rows: the per-tile partial sums of the MSE
+ * reduction and, when each (head, tile of 128 sampled rows) is split over up
+ * to 4 key ranges to fill a B200's 148 SMs, the unnormalised fp32 partial
+ * outputs and (base, sum) pairs of every split (B*H*tiles*splits*3*(d+2)*128
+ * floats). Depends only on the geometry and n_samples.
  */
 svg_status svg_profile_workspace_bytes(const svg_geom* geom, int32_t n_samples, size_t* bytes);
 

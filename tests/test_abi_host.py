@@ -129,7 +129,10 @@ def test_invalid_arguments_are_rejected_before_launch(svg):
     # profiling: too many samples, misaligned workspace, small workspace
     ws = ctypes.c_size_t()
     assert lib.svg_profile_workspace_bytes(ctypes.byref(g), 16, ctypes.byref(ws)) == svg.SVG_OK
-    assert ws.value == 2 * 2 * 1 * 4
+    # 2 CTAs (B*H = 2, one tile of samples) fill 148 SMs best with 4 key-range
+    # splits: per-tile errors (padded to 256 B), then the split partials
+    ctas, splits, d = 2, 4, 64
+    assert ws.value == 256 + ctas * splits * 3 * (d + 2) * 128 * 4
     assert lib.svg_profile_heads(ctypes.byref(g), 256, 256, 256, 256, 257, 256, None, 256,
                                  1 << 20, None) == svg.SVG_ERR_INVALID_ARG
     assert lib.svg_profile_heads(ctypes.byref(g), 256, 256, 256, 256, 16, 256, None, 260,

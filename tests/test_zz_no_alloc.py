@@ -6,7 +6,8 @@ latency-critical loop that cannot take cudaMalloc's implicit synchronisation,
 code with no allocator at hand). For them, svg_profile_heads_noalloc keeps the
 MSE partial sums in a fixed 256 KiB array inside the library. This test calls
 it through the C ABI twice in a row and checks both results against the
-workspace-taking svg_profile_heads on the same inputs. The file is named so
+workspace-taking svg_profile_heads on the same inputs (equal labels, MSE equal
+up to the rounding of a different summation order). The file is named so
 that pytest collects it last.
 """
 import numpy as np
@@ -51,7 +52,10 @@ def test_noalloc_matches_workspace_entry_point_twice(svg):
         lab_ref, mse_ref, lab, mse = _profile_both(svg, wl, seed_salt=call)
         assert torch.equal(lab, lab_ref)
         assert torch.all(torch.isfinite(mse))
-        np.testing.assert_allclose(mse.numpy(), mse_ref.numpy(), rtol=1e-6, atol=0)
+        # The workspace entry point may split each tile's key range over several
+        # CTAs to fill the GPU (the no-alloc one never does), so the fp32 sums
+        # are added in another order: equal labels, MSE equal to rounding.
+        np.testing.assert_allclose(mse.numpy(), mse_ref.numpy(), rtol=1e-3, atol=1e-9)
         assert list(lab.numpy()) == SI.planted_head_kinds(wl.replace(seed=wl.seed + call))
 
 

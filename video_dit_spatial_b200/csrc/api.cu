@@ -210,8 +210,8 @@ svg_status svg_profile_workspace_bytes(const svg_geom* geom, int32_t n_samples, 
   if (bytes == nullptr || n_samples < 1) return SVG_ERR_INVALID_ARG;
   const svg_status st = svg::check_geom(geom, false);
   if (st != SVG_OK) return st;
-  const size_t BH = static_cast<size_t>(geom->B) * geom->H;
-  *bytes = BH * 2 * static_cast<size_t>(svg::profile_tiles(n_samples)) * sizeof(float);
+  const Dims d = svg::make_dims(*geom);
+  *bytes = svg::profile_workspace_bytes(d, n_samples, svg::profile_splits(d, n_samples));
   return SVG_OK;
 }
 
@@ -235,7 +235,8 @@ svg_status svg_profile_heads(const svg_geom* geom, const svg_bf16* q, const svg_
   cudaError_t err;
   int* status = svg::device_status_word(&err);
   if (status == nullptr) return SVG_ERR_CUDA;
-  svg::ProfileArgs a{q, k, v, sample_idx, n_samples, labels, mse, static_cast<float*>(workspace)};
+  svg::ProfileArgs a{q,      k,   v, sample_idx, n_samples, labels, mse, static_cast<float*>(workspace),
+                     svg::profile_splits(d, n_samples)};
   if (svg::launch_profile(d, a, status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return SVG_ERR_CUDA;
   return SVG_OK;
@@ -252,14 +253,14 @@ svg_status svg_profile_heads_noalloc(const svg_geom* geom, const svg_bf16* q, co
   if (st != SVG_OK) return st;
   const Dims d = svg::make_dims(*geom);
   if (n_samples < 1 || n_samples > d.Nv) return SVG_ERR_INVALID_ARG;
-  size_t need = 0;
-  svg_profile_workspace_bytes(geom, n_samples, &need);
+  // one key range per (head, sample tile): only the per-tile errors
+  const size_t need = svg::profile_workspace_bytes(d, n_samples, 1);
   if (need > svg::profile_noalloc_scratch_bytes()) return SVG_ERR_CAPACITY;
   if ((st = svg::check_device()) != SVG_OK) return st;
   cudaError_t err;
   int* status = svg::device_status_word(&err);
   if (status == nullptr) return SVG_ERR_CUDA;
-  svg::ProfileArgs a{q, k, v, sample_idx, n_samples, labels, mse, nullptr};
+  svg::ProfileArgs a{q, k, v, sample_idx, n_samples, labels, mse, nullptr, 1};
   if (svg::launch_profile_noalloc(d, a, status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return SVG_ERR_CUDA;
   return SVG_OK;

@@ -114,9 +114,12 @@ struct ProfileArgs {
   int32_t n_samples;
   int8_t* labels;
   float* mse;
-  float* partial;  // [BH][2][n_tiles]
+  float* partial;    // the workspace: [BH][2][n_tiles] errors, then the split partials
+  int32_t n_splits;  // key-range splits per (head, sample tile), profile_splits()
 };
 int32_t profile_tiles(int32_t n_samples);
+int32_t profile_splits(const Dims& d, int32_t n_samples);
+size_t profile_workspace_bytes(const Dims& d, int32_t n_samples, int32_t n_splits);
 cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cudaStream_t stream);
 // Same launch with the partial sums in the module's fixed device scratch
 // (a.partial is ignored); see svg_profile_heads_noalloc.

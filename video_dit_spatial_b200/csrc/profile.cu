@@ -86,13 +86,18 @@ struct PCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
 
+// With n_splits > 1 each (head, sample tile) runs as n_splits CTAs over
+// consecutive ranges of key tiles; each writes its unnormalised accumulators
+// and (base, sum) pairs, and profile_combine_kernel merges them.
 struct __align__(64) ProfParams {
   CUtensorMap tm_k, tm_v;
   const svg_bf16* q;
   const int32_t* sample_idx;
   float* partial;  // [BH][2][n_tiles]
+  float* part_o;   // [BH][n_tiles][n_splits][3][D][128] (n_splits > 1)
+  float* part_ml;  // [BH][n_tiles][n_splits][3][2][128] (n_splits > 1)
   int* status;
-  int32_t n_samples, n_tiles;
+  int32_t n_samples, n_tiles, n_splits;
   int32_t N, Nv, T, P, s, w, nkt;
   float scale_log2;
 };
@@ -172,7 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
   const int warp = tid >> 5;
   const int tile = blockIdx.x;
   const int bh = blockIdx.y;
-  const int n = p.nkt;
+  // this CTA's key tiles: [j0, j0 + n)
+  const int split = blockIdx.z;
+  const int j0 = static_cast<int>(static_cast<long long>(p.nkt) * split / p.n_splits);
+  const int n = static_cast<int>(static_cast<long long>(p.nkt) * (split + 1) / p.n_splits) - j0;
 
   if (warp == 0) {
     tmem_alloc(&bar->tmem_base, C::kTmemCols);
@@ -244,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
           mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kKVPanel, &p.tm_k, &bar->k_full[st],
-                             pn * 64, j * kKeys, bh, keep);
+                             pn * 64, (j0 + j) * kKeys, bh, keep);
           k_issued = j + 1;
         }
         if (j >= 1) {
@@ -255,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
           mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kKVPanel, &p.tm_v, &bar->v_full[st],
-                             pn * 64, jv * kKeys, bh, keep);
+                             pn * 64, (j0 + jv) * kKeys, bh, keep);
           v_issued = jv + 1;
         }
       }
@@ -374,12 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     float m[3] = {-INFINITY, -INFINITY, -INFINITY};
     float l[3] = {0.0f, 0.0f, 0.0f};
     bool ok = true;
-    int fs0 = 0;  // start of the frame holding this thread's first key of the tile
+    // start of the frame holding this thread's first key of the tile
+    int fs0 = min(j0 * kKeys + c_base, p.Nv) / p.P * p.P;
     bool ps_zero[2] = {false, false};  // this warp's rows of P_spatial[buffer] hold zeros
     for (int j = 0; j < n; ++j) {
       const int sb = j & 1;
       const uint32_t s_col = lane_base + (sb ? C::kColS1 : C::kColS0);
-      const int k0 = j * kKeys + c_base;  // first key of this thread's half
+      const int k0 = (j0 + j) * kKeys + c_base;  // first key of this thread's half
       const int kvalid = max(0, min(kHalf, p.N - k0));
       const int k_end = k0 + kvalid;  // exclusive
       uint32_t bits[2] = {0u, 0u};    // allowed keys k0 + [0, 32): spatial, temporal
@@ -569,6 +578,41 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     for (int x = 0; x < 3; ++x) bar->xsum[half][x][row] = l[x];
     if (ok && n > 0) ok = mbar_wait(&bar->o_final, 0, abort_flag, p.status);
     softmax_sync();
+    if (p.n_splits > 1) {
+      // Partial results of this key range: the accumulators as they stand
+      // (relative to the running bases) and each row's (base, sum) pairs.
+      tc_fence_after();
+      const bool all_ok = __all_sync(0xffffffffu, ok);
+      const size_t cta = (static_cast<size_t>(bh) * p.n_tiles + tile) * p.n_splits + split;
+      float* po = p.part_o + cta * 3 * D * kRows;
+#pragma unroll
+      for (int x = 0; x < 3; ++x) {
+        const uint32_t ocol =
+            lane_base + (x == 0 ? C::kColOF : (x == 1 ? C::kColOS : C::kColOT)) + half * (D / 2);
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) {
+          uint32_t o[32];
+          if (all_ok && n > 0) {
+            tmem_ld_32x32b_x32(ocol + ch * 32, o);
+            tmem_ld_wait();
+            reg_fence(o);
+          }
+          const int c0 = half * (D / 2) + ch * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            po[(static_cast<size_t>(x) * D + c0 + i) * kRows + row] =
+                all_ok && n > 0 && bar->xsum[0][x][row] + bar->xsum[1][x][row] > 0.0f
+                    ? u2f(o[i])
+                    : 0.0f;
+        }
+        if (half == 0) {
+          float* pml = p.part_ml + (cta * 3 + x) * 2 * kRows;
+          const float L = bar->xsum[0][x][row] + bar->xsum[1][x][row];
+          pml[row] = all_ok ? (L > 0.0f ? m[x] : -INFINITY) : __int_as_float(0x7fc00000);
+          pml[kRows + row] = all_ok ? L : __int_as_float(0x7fc00000);
+        }
+      }
+    } else {
     float inv[3];
 #pragma unroll
     for (int x = 0; x < 3; ++x) {
@@ -612,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       p.partial[(static_cast<size_t>(bh) * 2 + x) * p.n_tiles + tile] =
           *abort_flag ? __int_as_float(0x7fc00000) : acc;
     }
+    }
   }
 
   tc_fence_before();
@@ -619,6 +664,68 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Merges the key-range partials of one (head, sample tile): per row and
+// softmax, weights 2^(m_s - max m) put the splits on one base; the merged
+// outputs give the row's squared errors, which are added over rows in a fixed
+// order into the same per-tile slot the unsplit kernel fills.
+template <int D>
+__global__ void __launch_bounds__(kRows) profile_combine_kernel(const __grid_constant__ ProfParams p) {
+  __shared__ float red[2][kRows];
+  const int tile = blockIdx.x, bh = blockIdx.y, row = threadIdx.x;
+  const int S = p.n_splits;
+  const size_t cta0 = (static_cast<size_t>(bh) * p.n_tiles + tile) * S;
+  const int si = tile * kRows + row;
+  bool valid = si < p.n_samples;
+  if (valid) {
+    const int r = __ldg(p.sample_idx + si);
+    valid = r >= 0 && r < p.Nv;
+  }
+  float err[2] = {0.0f, 0.0f};
+  bool aborted = false;  // a split that gave up writes NaN pairs
+  for (int sp = 0; sp < S; ++sp)
+    for (int x = 0; x < 3; ++x)
+      aborted |= isnan(p.part_ml[((cta0 + sp) * 3 + x) * 2 * kRows + row]);
+  if (valid && !aborted) {
+    float mx[3] = {-INFINITY, -INFINITY, -INFINITY};
+    for (int sp = 0; sp < S; ++sp)
+      for (int x = 0; x < 3; ++x)
+        mx[x] = fmaxf(mx[x], p.part_ml[((cta0 + sp) * 3 + x) * 2 * kRows + row]);
+    float inv[3];
+    for (int x = 0; x < 3; ++x) {
+      float L = 0.0f;
+      for (int sp = 0; sp < S; ++sp) {
+        const float* ml = p.part_ml + ((cta0 + sp) * 3 + x) * 2 * kRows;
+        if (ml[row] != -INFINITY) L += exp2f(ml[row] - mx[x]) * ml[kRows + row];
+      }
+      inv[x] = L > 0.0f ? 1.0f / L : 0.0f;
+    }
+    for (int c = 0; c < D; ++c) {
+      float o[3] = {0.0f, 0.0f, 0.0f};
+      for (int sp = 0; sp < S; ++sp) {
+        for (int x = 0; x < 3; ++x) {
+          const float mv = p.part_ml[((cta0 + sp) * 3 + x) * 2 * kRows + row];
+          if (mv == -INFINITY) continue;
+          const float w = exp2f(mv - mx[x]);
+          o[x] = fmaf(w, p.part_o[(((cta0 + sp) * 3 + x) * D + c) * kRows + row], o[x]);
+        }
+      }
+      const float oF = o[0] * inv[0];
+      for (int x = 0; x < 2; ++x) {
+        const float dlt = o[1 + x] * inv[1 + x] - oF;
+        err[x] = fmaf(dlt, dlt, err[x]);
+      }
+    }
+  }
+  red[0][row] = aborted ? __int_as_float(0x7fc00000) : err[0];
+  red[1][row] = aborted ? __int_as_float(0x7fc00000) : err[1];
+  __syncthreads();
+  if (row < 2) {
+    float acc = 0.0f;
+    for (int i = 0; i < kRows; ++i) acc += red[row][i];
+    p.partial[(static_cast<size_t>(bh) * 2 + row) * p.n_tiles + tile] = acc;
   }
 }
 
@@ -649,9 +756,14 @@ cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, flo
   auto kern = profile_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(pp.n_tiles, d.BH), kThreads, C::kSmem, stream>>>(pp);
+  kern<<<dim3(pp.n_tiles, d.BH, pp.n_splits), kThreads, C::kSmem, stream>>>(pp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (pp.n_splits > 1) {
+    profile_combine_kernel<D><<<dim3(pp.n_tiles, d.BH), kRows, 0, stream>>>(pp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const float inv = 1.0f / (static_cast<float>(pp.n_samples) * static_cast<float>(D));
   profile_finalize_kernel<<<(d.BH + 127) / 128, 128, 0, stream>>>(pp.partial, d.BH, pp.n_tiles,
                                                                   inv, labels, mse);
@@ -661,6 +773,37 @@ cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, flo
 }  // namespace
 
 int32_t profile_tiles(int32_t n_samples) { return (n_samples + kRows - 1) / kRows; }
+
+// Key-range splits per (head, sample tile): the count in 1..4 (never more than
+// the key tiles) that fills the last wave best on a B200's 148 SMs, one CTA
+// each; ties go to fewer splits.
+int32_t profile_splits(const Dims& d, int32_t n_samples) {
+  constexpr int64_t kSMs = 148;
+  const int64_t ctas = static_cast<int64_t>(d.BH) * profile_tiles(n_samples);
+  const int32_t nkt = (d.N + kKeys - 1) / kKeys;
+  int32_t best = 1;
+  double best_fill = 0.0;
+  for (int32_t sp = 1; sp <= 4 && sp <= nkt; ++sp) {
+    const int64_t c = ctas * sp;
+    const double fill = static_cast<double>(c) / static_cast<double>((c + kSMs - 1) / kSMs * kSMs);
+    if (fill > best_fill + 1e-9) {
+      best = sp;
+      best_fill = fill;
+    }
+  }
+  return best;
+}
+
+size_t profile_workspace_bytes(const Dims& d, int32_t n_samples, int32_t n_splits) {
+  const size_t ctas = static_cast<size_t>(d.BH) * profile_tiles(n_samples);
+  size_t bytes = ctas * 2 * sizeof(float);  // per-tile errors
+  if (n_splits > 1) {
+    bytes = (bytes + 255) / 256 * 256;
+    bytes += ctas * n_splits * 3 * static_cast<size_t>(d.d) * kRows * sizeof(float);
+    bytes += ctas * n_splits * 3 * 2 * kRows * sizeof(float);
+  }
+  return bytes;
+}
 
 // ---------------------------------------------------------------------------
 // Fixed scratch for svg_profile_heads_noalloc: the per-tile partial sums live
@@ -705,6 +848,7 @@ cudaError_t launch_profile_noalloc(const Dims& d, const ProfileArgs& a, int* sta
   if (e != cudaSuccess) return e;
   ProfileArgs args = a;
   args.partial = scratch;
+  args.n_splits = 1;
   return launch_profile(d, args, status, stream);
 }
 
@@ -717,6 +861,14 @@ cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cud
   pp.q = a.q;
   pp.sample_idx = a.sample_idx;
   pp.partial = a.partial;
+  pp.n_splits = a.n_splits;
+  if (a.n_splits > 1) {
+    const size_t ctas = static_cast<size_t>(d.BH) * profile_tiles(a.n_samples);
+    uint8_t* base = reinterpret_cast<uint8_t*>(a.partial);
+    const size_t off_o = (ctas * 2 * sizeof(float) + 255) / 256 * 256;
+    pp.part_o = reinterpret_cast<float*>(base + off_o);
+    pp.part_ml = pp.part_o + ctas * a.n_splits * 3 * static_cast<size_t>(d.d) * kRows;
+  }
   pp.status = status;
   pp.n_samples = a.n_samples;
   pp.n_tiles = profile_tiles(a.n_samples);
