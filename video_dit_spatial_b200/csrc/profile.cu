@@ -383,30 +383,48 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     float l[3] = {0.0f, 0.0f, 0.0f};
     bool ok = true;
     // start of the frame holding this thread's first key of the tile
-    int fs0 = min(j0 * kKeys + c_base, p.Nv) / p.P * p.P;
+    // Allowed-key bits of a half tile: text keys, the spatial run, and the
+    // temporal run of each frame overlapping the half tile. r0 = k0 mod P; with
+    // P >= 32 at most two frames overlap 32 keys and the bits need no branch,
+    // so the next tile's bits are computed in the shadow of this tile's
+    // exponentials.
+    auto tile_bits = [&](int jt, int r0, uint32_t (&b)[2]) {
+      const int k0 = (j0 + jt) * kKeys + c_base;
+      const int kvalid = max(0, min(kHalf, p.N - k0));
+      const int v_end = min(k0 + kvalid, p.Nv);
+      const uint32_t text = bit_range32(p.Nv - k0, kvalid);
+      uint32_t bt = 0u;
+      if (p.P >= kHalf) {
+        const int fs = k0 - r0;
+        bt = bit_range32(fs + t_lo - k0, min(fs + t_hi + 1, v_end) - k0) |
+             bit_range32(fs + p.P + t_lo - k0, min(fs + p.P + t_hi + 1, v_end) - k0);
+      } else {
+        for (int fs = k0 - r0; fs < v_end; fs += p.P)
+          bt |= bit_range32(fs + t_lo - k0, min(fs + t_hi + 1, v_end) - k0);
+      }
+      const bool any = row_valid && kvalid > 0;
+      b[0] = any ? text | bit_range32(s_lo - k0, min(s_hi, v_end) - k0) : 0u;
+      b[1] = any ? text | bt : 0u;
+    };
+    auto next_r0 = [&](int r0) {  // (k0 + 64) mod P from k0 mod P
+      r0 += kKeys;
+      if (p.P >= kKeys / 2) {
+        r0 = r0 >= p.P ? r0 - p.P : r0;
+        r0 = r0 >= p.P ? r0 - p.P : r0;
+      } else {
+        r0 %= p.P;
+      }
+      return r0;
+    };
+    int r0 = (j0 * kKeys + c_base) % p.P;
+    uint32_t bits[2];  // allowed keys k0 + [0, 32) of this tile: spatial, temporal
+    tile_bits(0, r0, bits);
     bool ps_zero[2] = {false, false};  // this warp's rows of P_spatial[buffer] hold zeros
     for (int j = 0; j < n; ++j) {
       const int sb = j & 1;
       const uint32_t s_col = lane_base + (sb ? C::kColS1 : C::kColS0);
       const int k0 = (j0 + j) * kKeys + c_base;  // first key of this thread's half
       const int kvalid = max(0, min(kHalf, p.N - k0));
-      const int k_end = k0 + kvalid;  // exclusive
-      uint32_t bits[2] = {0u, 0u};    // allowed keys k0 + [0, 32): spatial, temporal
-      if (row_valid && kvalid > 0) {
-        if (k_end > p.Nv) {
-          const uint32_t text = bit_range32(max(p.Nv, k0) - k0, kvalid);
-          bits[0] = bits[1] = text;
-        }
-        if (k0 < p.Nv) {
-          const int v_end = min(k_end, p.Nv);
-          bits[0] |= bit_range32(max(s_lo, k0) - k0, min(s_hi, v_end) - k0);
-          // frames overlapping the half tile; fs0 tracks the start of the frame
-          // holding k0 across tiles
-          while (fs0 + p.P <= k0) fs0 += p.P;
-          for (int fs = fs0; fs < v_end; fs += p.P)
-            bits[1] |= bit_range32(fs + t_lo - k0, min(fs + t_hi + 1, v_end) - k0);
-        }
-      }
 
       if (ok && !mbar_wait(&bar->s_full[sb], (j >> 1) & 1, abort_flag, p.status)) ok = false;
       // Both warps of a pair must take the same path through pair_sync (an
@@ -490,6 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       }
       tmem_st_32x32b_x16(s_col + half * (kHalf / 2), pkF);
       float sum[3] = {sF0 + sF1, 0.0f, 0.0f};
+      uint32_t next_bits[2];
+      const int r0_next = next_r0(r0);
+      tile_bits(j + 1, r0_next, next_bits);
       // masked probabilities: P_X = P_full * 2^(u_full - u_X) on allowed keys,
       // unless the masked base is so far below the full one that the full
       // probabilities could flush to zero; those rows (rare) take the masked
@@ -571,6 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
       }
       tc_fence_before();
       mbar_arrive(&bar->p_full[sb]);
+      bits[0] = next_bits[0];
+      bits[1] = next_bits[1];
+      r0 = r0_next;
     }
 
     // ---- per-row squared errors over this half's d/2 channels
