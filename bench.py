@@ -369,8 +369,12 @@ def main():
     clock_info = clocks.stop() if clocks else None
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
     # profile, finalize, 2 masks, attention, plus the layout passes: permute_qkv and
-    # unpermute (explicit), permute of K and V (fused), none (gathered)
-    gpu_launches = {"explicit": 7, "fused": 6, "gathered": 5}[layout] * args.steps
+    # unpermute (explicit), permute of K and V (fused), none (gathered); plus the
+    # profiling combine kernel when the key ranges are split (a workspace larger
+    # than the per-tile sums)
+    tiles = (wl.n_samples + 127) // 128
+    split = svg.svg_profile_workspace_bytes(g, wl.n_samples) > wl.B * wl.H * 2 * tiles * 4
+    gpu_launches = ({"explicit": 7, "fused": 6, "gathered": 5}[layout] + int(split)) * args.steps
 
     # per-kernel timing (events on the launch stream), then the dense baseline
     def time_fn(fn, reps):
