@@ -695,10 +695,15 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
 // softmax, weights 2^(m_s - max m) put the splits on one base; the merged
 // outputs give the row's squared errors, which are added over rows in a fixed
 // order into the same per-tile slot the unsplit kernel fills.
+constexpr int kCombineQuarters = 4;  // threads per row, each a quarter of the channels
+constexpr int kMaxSplits = 4;
+
 template <int D>
-__global__ void __launch_bounds__(kRows) profile_combine_kernel(const __grid_constant__ ProfParams p) {
-  __shared__ float red[2][kRows];
-  const int tile = blockIdx.x, bh = blockIdx.y, row = threadIdx.x;
+__global__ void __launch_bounds__(kRows * kCombineQuarters)
+    profile_combine_kernel(const __grid_constant__ ProfParams p) {
+  __shared__ float red[2][kCombineQuarters][kRows];
+  const int tile = blockIdx.x, bh = blockIdx.y;
+  const int row = threadIdx.x % kRows, quarter = threadIdx.x / kRows;
   const int S = p.n_splits;
   const size_t cta0 = (static_cast<size_t>(bh) * p.n_tiles + tile) * S;
   const int si = tile * kRows + row;
@@ -707,49 +712,66 @@ __global__ void __launch_bounds__(kRows) profile_combine_kernel(const __grid_con
     const int r = __ldg(p.sample_idx + si);
     valid = r >= 0 && r < p.Nv;
   }
-  float err[2] = {0.0f, 0.0f};
+  // per split and softmax: weight 2^(m_s - max m) of the split's accumulator
+  float m_s[kMaxSplits][3], l_s[kMaxSplits][3];
   bool aborted = false;  // a split that gave up writes NaN pairs
-  for (int sp = 0; sp < S; ++sp)
-    for (int x = 0; x < 3; ++x)
-      aborted |= isnan(p.part_ml[((cta0 + sp) * 3 + x) * 2 * kRows + row]);
-  if (valid && !aborted) {
-    float mx[3] = {-INFINITY, -INFINITY, -INFINITY};
-    for (int sp = 0; sp < S; ++sp)
-      for (int x = 0; x < 3; ++x)
-        mx[x] = fmaxf(mx[x], p.part_ml[((cta0 + sp) * 3 + x) * 2 * kRows + row]);
-    float inv[3];
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplits; ++sp)
+#pragma unroll
     for (int x = 0; x < 3; ++x) {
-      float L = 0.0f;
-      for (int sp = 0; sp < S; ++sp) {
+      m_s[sp][x] = -INFINITY;
+      l_s[sp][x] = 0.0f;
+      if (sp < S) {
         const float* ml = p.part_ml + ((cta0 + sp) * 3 + x) * 2 * kRows;
-        if (ml[row] != -INFINITY) L += exp2f(ml[row] - mx[x]) * ml[kRows + row];
+        m_s[sp][x] = ml[row];
+        l_s[sp][x] = ml[kRows + row];
+        aborted |= isnan(m_s[sp][x]) || isnan(l_s[sp][x]);
       }
-      inv[x] = L > 0.0f ? 1.0f / L : 0.0f;
     }
-    for (int c = 0; c < D; ++c) {
+  float w[kMaxSplits][3], inv[3];
+#pragma unroll
+  for (int x = 0; x < 3; ++x) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) mx = fmaxf(mx, m_s[sp][x]);
+    float L = 0.0f;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+      w[sp][x] = m_s[sp][x] == -INFINITY ? 0.0f : exp2f(m_s[sp][x] - mx);
+      L = fmaf(w[sp][x], l_s[sp][x], L);
+    }
+    inv[x] = L > 0.0f ? 1.0f / L : 0.0f;
+  }
+  float err[2] = {0.0f, 0.0f};
+  if (valid && !aborted) {
+    for (int c = quarter * (D / kCombineQuarters); c < (quarter + 1) * (D / kCombineQuarters);
+         ++c) {
       float o[3] = {0.0f, 0.0f, 0.0f};
-      for (int sp = 0; sp < S; ++sp) {
-        for (int x = 0; x < 3; ++x) {
-          const float mv = p.part_ml[((cta0 + sp) * 3 + x) * 2 * kRows + row];
-          if (mv == -INFINITY) continue;
-          const float w = exp2f(mv - mx[x]);
-          o[x] = fmaf(w, p.part_o[(((cta0 + sp) * 3 + x) * D + c) * kRows + row], o[x]);
-        }
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplits; ++sp) {
+        if (sp >= S) break;
+#pragma unroll
+        for (int x = 0; x < 3; ++x)
+          o[x] = fmaf(w[sp][x], __ldg(p.part_o + (((cta0 + sp) * 3 + x) * D + c) * kRows + row),
+                      o[x]);
       }
       const float oF = o[0] * inv[0];
+#pragma unroll
       for (int x = 0; x < 2; ++x) {
         const float dlt = o[1 + x] * inv[1 + x] - oF;
         err[x] = fmaf(dlt, dlt, err[x]);
       }
     }
   }
-  red[0][row] = aborted ? __int_as_float(0x7fc00000) : err[0];
-  red[1][row] = aborted ? __int_as_float(0x7fc00000) : err[1];
+  red[0][quarter][row] = aborted ? __int_as_float(0x7fc00000) : err[0];
+  red[1][quarter][row] = aborted ? __int_as_float(0x7fc00000) : err[1];
   __syncthreads();
-  if (row < 2) {
+  if (threadIdx.x < 2) {
+    const int x = threadIdx.x;
     float acc = 0.0f;
-    for (int i = 0; i < kRows; ++i) acc += red[row][i];
-    p.partial[(static_cast<size_t>(bh) * 2 + row) * p.n_tiles + tile] = acc;
+    for (int i = 0; i < kRows; ++i)
+      for (int q = 0; q < kCombineQuarters; ++q) acc += red[x][q][i];
+    p.partial[(static_cast<size_t>(bh) * 2 + x) * p.n_tiles + tile] = acc;
   }
 }
 
@@ -784,7 +806,8 @@ cudaError_t launch_impl(const Dims& d, const ProfParams& pp, int8_t* labels, flo
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (pp.n_splits > 1) {
-    profile_combine_kernel<D><<<dim3(pp.n_tiles, d.BH), kRows, 0, stream>>>(pp);
+    profile_combine_kernel<D>
+        <<<dim3(pp.n_tiles, d.BH), kRows * kCombineQuarters, 0, stream>>>(pp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -807,7 +830,7 @@ int32_t profile_splits(const Dims& d, int32_t n_samples) {
   const int32_t nkt = (d.N + kKeys - 1) / kKeys;
   int32_t best = 1;
   double best_fill = 0.0;
-  for (int32_t sp = 1; sp <= 4 && sp <= nkt; ++sp) {
+  for (int32_t sp = 1; sp <= kMaxSplits && sp <= nkt; ++sp) {
     const int64_t c = ctas * sp;
     const double fill = static_cast<double>(c) / static_cast<double>((c + kSMs - 1) / kSMs * kSMs);
     if (fill > best_fill + 1e-9) {
