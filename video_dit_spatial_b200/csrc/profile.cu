@@ -604,9 +604,12 @@ __global__ void __launch_bounds__(kThreads, 1) profile_kernel(const __grid_const
     softmax_sync();
     if (p.n_splits > 1) {
       // Partial results of this key range: the accumulators as they stand
-      // (relative to the running bases) and each row's (base, sum) pairs.
+      // (relative to the running bases) and each row's (base, sum) pairs. A
+      // failure anywhere in the CTA turns all its pairs into NaN.
+      if (!__all_sync(0xffffffffu, ok)) atomicOr(&bar->abort_flag, 1);
+      softmax_sync();
       tc_fence_after();
-      const bool all_ok = __all_sync(0xffffffffu, ok);
+      const bool all_ok = *abort_flag == 0;
       const size_t cta = (static_cast<size_t>(bh) * p.n_tiles + tile) * p.n_splits + split;
       float* po = p.part_o + cta * 3 * D * kRows;
 #pragma unroll
