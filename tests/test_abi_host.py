@@ -142,6 +142,42 @@ def test_invalid_arguments_are_rejected_before_launch(svg):
     assert lib.svg_selftest_wait_timeout(0, None) == svg.SVG_ERR_INVALID_ARG
 
 
+def _expected_splits(ctas, nkt, sms=148):
+    """The documented rule: the split count in 1..4 (at most the key tiles) whose
+    CTAs fill the last wave of 148 SMs best; ties go to fewer splits."""
+    best, best_fill = 1, 0.0
+    for sp in range(1, min(4, nkt) + 1):
+        c = ctas * sp
+        fill = c / (-(-c // sms) * sms)
+        if fill > best_fill + 1e-9:
+            best, best_fill = sp, fill
+    return best
+
+
+@pytest.mark.parametrize("name", ["cogvideox15_B1_H48_d64_T11_P4080_L226",
+                                  "hunyuan_B1_H24_d128_T33_P3600_L256",
+                                  "long_B2_H8_d128_T64_P3600_L256", "sweep_s2_w256",
+                                  "tiny_B1_H2_d64_T4_P64"])
+def test_profile_workspace_follows_the_split_rule(svg, name):
+    import svg_inputs as SI
+    wl = SI.WORKLOADS[name]
+    g = svg.Geom.from_workload(wl)
+    S = wl.n_samples
+    tiles = -(-S // 128)
+    ctas = wl.B * wl.H * tiles
+    nkt = -(-wl.N // 64)
+    sp = _expected_splits(ctas, nkt)
+    want = ctas * 2 * 4
+    if sp > 1:
+        want = -(-want // 256) * 256 + ctas * sp * 3 * (wl.d + 2) * 128 * 4
+    assert svg.svg_profile_workspace_bytes(g, S) == want
+    # the configurations the benchmark runs split as documented
+    expected = {"hunyuan_B1_H24_d128_T33_P3600_L256": 3, "long_B2_H8_d128_T64_P3600_L256": 4,
+                "cogvideox15_B1_H48_d64_T11_P4080_L226": 3}
+    if name in expected:
+        assert sp == expected[name]
+
+
 def test_no_device_reports_cuda_error(svg):
     import torch
     if torch.cuda.is_available():
