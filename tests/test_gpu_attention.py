@@ -104,6 +104,32 @@ def test_dense_baseline_is_full_attention(svg, case):
     status_clean()
 
 
+@pytest.mark.parametrize("T,P,L,d,bq,bk", [(6, 50, 10, 64, 64, 64), (5, 100, 37, 128, 128, 128),
+                                           (3, 40, 0, 128, 128, 64)])
+def test_full_width_bands_equal_the_dense_run(svg, T, P, L, d, bq, bk):
+    # With s >= T-1 and w >= P-1 both masks list every key block: the spatial CSR is the
+    # dense one, so spatial heads must give the dense run's bits, and temporal heads
+    # (position-major, the same keys in another order) the oracle's full attention.
+    N = T * P + L
+    g = svg.Geom(1, 2, T, P, L, d, bq, bk, T - 1, P - 1, 1.0 / np.sqrt(d))
+    q, k, v = (rand_bf16((1, 2, N, d), seed=900 + i) for i in range(3))
+    layer = _layer(svg, g)
+    layer.build_masks()
+    layer.labels.copy_(torch.tensor([0, 1], dtype=torch.int8))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o = torch.empty_like(qd)
+    od = torch.empty_like(qd)
+    layer.attend(qd, kd, vd, o)
+    layer.dense(qd, kd, vd, od)
+    torch.cuda.synchronize()
+    assert torch.equal(layer.masks[0].row_ptr, layer.dense_mask.row_ptr)
+    assert torch.equal(o[0, 0].view(torch.int16), od[0, 0].view(torch.int16))
+    want, _ = O.masked_attention_rows(to_f64(q[0, 1]), to_f64(k[0, 1]), to_f64(v[0, 1]),
+                                      np.arange(N), None, 1.0 / np.sqrt(d))
+    assert_close(to_f64(o[0, 1]), want, "temporal head, full-width band")
+    status_clean()
+
+
 def test_empty_csr_rows_give_zero(svg):
     T, P, L, d = 2, 128, 0, 128
     N = T * P

@@ -31,6 +31,8 @@ SMALL_GEOMS = [
     (1, 300, 1, 64, 64, 0, 0),
     (40, 3, 0, 128, 128, 3, 1),
     (7, 129, 129, 64, 64, 1, 64),
+    (6, 50, 10, 64, 64, 5, 49),     # s = T-1, w = P-1: both masks are every block
+    (3, 40, 0, 128, 64, 7, 100),    # bands wider than the grid
 ]
 
 
