@@ -131,7 +131,8 @@ svg_status svg_profile_workspace_bytes(const svg_geom* geom, int32_t n_samples, 
  *   labels       device int8 [B*H], out.
  *   mse          device float [B*H*2] out ({spatial, temporal} per head), or NULL.
  *   workspace    device, >= svg_profile_workspace_bytes(...), 256-byte aligned.
- * Deterministic: fixed-order reductions, no atomics in the arithmetic.
+ * Deterministic for a given geometry and n_samples: fixed-order reductions,
+ * no atomics in the arithmetic.
  * Errors: INVALID_ARG, UNSUPPORTED, CAPACITY (workspace too small), CUDA.
  * A sample index outside [0, T*P) sets the device bounds bit (row skipped).
  */
@@ -151,10 +152,14 @@ svg_status svg_profile_heads(const svg_geom* geom, const svg_bf16* q, const svg_
  * arguments as svg_profile_heads minus the workspace and keeps the MSE
  * partial sums in a fixed array inside the library instead; it calls no
  * cudaMalloc, cudaFree or other allocating routine.
- *   Limit      the partial sums need B*H*2*ceil(n_samples/128)*4 bytes
- *              (svg_profile_workspace_bytes); more than 256 KiB (that is,
- *              B*H*ceil(n_samples/128) > 32768) returns SVG_ERR_CAPACITY
- *              before anything is launched.
+ *   Limit      the partial sums need B*H*2*ceil(n_samples/128)*4 bytes (one
+ *              key range per tile of 128 sampled rows: unlike
+ *              svg_profile_heads it never splits the key range); more than
+ *              256 KiB (that is, B*H*ceil(n_samples/128) > 32768) returns
+ *              SVG_ERR_CAPACITY before anything is launched.
+ *   Results    the same labels as svg_profile_heads; the MSE values agree up
+ *              to the rounding of the summation order when svg_profile_heads
+ *              splits the key ranges.
  *   Memory     every GPU that loads the library holds the 256 KiB array
  *              until the process exits.
  *   Set-up     the first call on a device looks up that device's copy of
