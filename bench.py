@@ -478,7 +478,9 @@ def main():
         cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"fp64 oracle attention output of 96 query rows x 2 heads (one spatial, "
                          f"one temporal) of {wl.name}, with their block-mask rows",
-               "seconds": secs}
+               "seconds": secs,
+               # labelled extrapolation: the sample's rate over the layer's computed pairs
+               "extrapolated_layer_hours": attn_flops / (fl / secs) / 3600.0}
 
     if rank == 0:
         line = {
