@@ -194,3 +194,17 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(OSError):
         m.load()
+
+
+def test_python_binding_rejects_host_tensors():
+    # A host address handed to a kernel would fault on the device: the binding
+    # refuses CPU tensors before anything reaches the library.
+    import torch
+    import video_dit_spatial_b200 as m
+    g = m.Geom(1, 1, 2, 4, 0, 64, 64, 64, 0, 0, 0.125)
+    x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="device buffers"):
+        m.svg_permute(g, x, torch.zeros_like(x))
+    with pytest.raises(ValueError, match="device buffers"):
+        m._ptr(x.transpose(2, 3))
+    assert m._ptr(None) is None and m._ptr(1234) == 1234

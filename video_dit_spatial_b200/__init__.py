@@ -117,10 +117,17 @@ def load() -> ctypes.CDLL:
 
 
 def _ptr(x) -> Optional[int]:
+    """Device address of a buffer argument: None, a plain integer address, or a
+    tensor. A tensor must live on a CUDA device and be contiguous: the kernels
+    read dense row-major buffers, and a host address would fault on the device."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if not x.is_cuda:
+        raise ValueError(f"libsvg takes device buffers, got a tensor on {x.device}")
+    if not x.is_contiguous():
+        raise ValueError("libsvg takes contiguous buffers, got a strided view")
     return x.data_ptr()
 
 
