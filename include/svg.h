@@ -164,7 +164,11 @@ svg_status svg_profile_heads(const svg_geom* geom, const svg_bf16* q, const svg_
  *              until the process exits.
  *   Set-up     the first call on a device looks up that device's copy of
  *              the array (cudaGetSymbolAddress) with the device current;
- *              make that first call before any stream capture.
+ *              make that first call before any stream capture. A device
+ *              reset (cudaDeviceReset) loads the library's device code again
+ *              at another address: the next call notices the new context and
+ *              looks the address up again, so after a reset, too, make one
+ *              call before any stream capture.
  *   Sharing    all calls share the one array and it keeps the last call's
  *              contents (every slot is written before it is read, so no
  *              clearing is needed); calls that overlap on the GPU (e.g. on
@@ -287,15 +291,6 @@ svg_status svg_get_device_status(svg_stream_t stream, int32_t* bits);
  * timeout status bit and the kernel returns normally; no fault, trap or hang.
  */
 svg_status svg_selftest_wait_timeout(int64_t limit_cycles, svg_stream_t stream);
-
-/* ---------------------------------------------------------------------------
- * svg_selftest_exp2 -- applies the kernels' FMA-pipe 2^y evaluation (range
- * reduction to y = n + f, minimax cubic for 2^f, exponent-field scaling) to
- * in[0..n) and writes out[0..n); device float arrays, n in [1, 2^31]. Lets a
- * test bound its error against exact 2^y. Inputs below -125 are clamped to
- * -125 (the result is then a value in (0, 2^-124]).
- */
-svg_status svg_selftest_exp2(const float* in, float* out, int64_t n, svg_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* svg_status_string(svg_status status);

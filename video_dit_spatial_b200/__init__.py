@@ -36,7 +36,6 @@ EXPORTED = [
     "svg_mask_nnz", "svg_build_block_mask", "svg_profile_workspace_bytes",
     "svg_profile_heads", "svg_profile_heads_noalloc", "svg_permute", "svg_unpermute", "svg_permute_qkv",
     "svg_sparse_attention", "svg_sparse_attention_fused", "svg_get_device_status", "svg_selftest_wait_timeout",
-    "svg_selftest_exp2",
     "svg_status_string", "svg_version",
 ]
 
@@ -104,7 +103,6 @@ def load() -> ctypes.CDLL:
         "svg_sparse_attention_fused": [_c_geom_p] + [_vp] * 13,
         "svg_get_device_status": [_vp, ctypes.POINTER(_i32)],
         "svg_selftest_wait_timeout": [_i64, _vp],
-        "svg_selftest_exp2": [_vp, _vp, _i64, _vp],
         "svg_status_string": [_i32],
         "svg_version": [],
     }
@@ -231,11 +229,6 @@ def svg_get_device_status(stream=None):
     bits = _i32(0)
     st = load().svg_get_device_status(_stream(stream), ctypes.byref(bits))
     return st, bits.value
-
-
-def svg_selftest_exp2(inp, out, stream=None) -> None:
-    _check("svg_selftest_exp2", load().svg_selftest_exp2(_ptr(inp), _ptr(out), inp.numel(),
-                                                         _stream(stream)))
 
 
 def svg_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:

@@ -21,7 +21,11 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 int* g_status_ptr[kMaxDevices] = {};
+void* g_status_ctx[kMaxDevices] = {};  // context the cached address belongs to
 int g_is_sm100[kMaxDevices] = {};  // 0 unknown, 1 yes, -1 no
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn g_ctx_get = nullptr;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -40,6 +44,18 @@ EncodeTiledFn encode_fn() {
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   }
   return g_encode;
+}
+
+CtxGetCurrentFn ctx_get_fn() {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_ctx_get == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get = reinterpret_cast<CtxGetCurrentFn>(fn);
+  }
+  return g_ctx_get;
 }
 
 inline bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -114,16 +130,31 @@ Dims make_dims(const svg_geom& g) {
   return d;
 }
 
+void* current_context() {
+  CtxGetCurrentFn get = ctx_get_fn();
+  CUcontext c = nullptr;
+  if (get == nullptr || get(&c) != CUDA_SUCCESS) return nullptr;
+  return static_cast<void*>(c);
+}
+
 int* device_status_word(cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_status_ptr[dev] == nullptr) {
+  // A device reset tears the context down and the module is loaded again into
+  // the next one, at a new address: look it up again whenever the context changes.
+  if (g_status_ptr[dev] == nullptr || ctx == nullptr || g_status_ctx[dev] != ctx) {
     void* ptr = nullptr;
-    *err = cudaGetSymbolAddress(&ptr, g_device_status);
+    *err = cudaGetSymbolAddress(&ptr, g_device_status);  // initialises the context if needed
     if (*err != cudaSuccess) return nullptr;
     g_status_ptr[dev] = static_cast<int*>(ptr);
+    g_status_ctx[dev] = current_context();
   }
   return g_status_ptr[dev];
 }
@@ -423,34 +454,11 @@ __global__ void wait_selftest_kernel(long long limit, int* status) {
 }
 }  // namespace
 
-__global__ void exp2_selftest_kernel(const float* __restrict__ in, float* __restrict__ out,
-                                     int64_t n) {
-  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    exp2_poly2(out[i], out[i + 1], in[i], in[i + 1]);
-  } else if (i < n) {
-    float dummy;
-    exp2_poly2(out[i], dummy, in[i], 0.0f);
-  }
-}
-
 cudaError_t launch_wait_selftest(long long limit_cycles, int* status, cudaStream_t stream) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_cycles, status);
   return cudaGetLastError();
 }
 }  // namespace svg
-
-extern "C" svg_status svg_selftest_exp2(const float* in, float* out, int64_t n,
-                                        svg_stream_t stream) {
-  if (in == nullptr || out == nullptr || n < 1 || n > (static_cast<int64_t>(1) << 31))
-    return SVG_ERR_INVALID_ARG;
-  svg_status st = svg::check_device();
-  if (st != SVG_OK) return st;
-  const int64_t pairs = (n + 1) / 2;
-  svg::exp2_selftest_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0,
-                              static_cast<cudaStream_t>(stream)>>>(in, out, n);
-  return cudaGetLastError() == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
-}
 
 extern "C" svg_status svg_selftest_wait_timeout(int64_t limit_cycles, svg_stream_t stream) {
   if (limit_cycles < 1 || limit_cycles > (static_cast<int64_t>(1) << 31)) return SVG_ERR_INVALID_ARG;

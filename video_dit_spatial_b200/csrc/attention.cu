@@ -399,11 +399,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kPairThreads = 384;
 constexpr int kPairProducerWarp = 8;
 constexpr int kPairMmaWarp = 9;
-// One exp2 pair in kPairEmuEvery on the FMA pipe (0 = all on MUFU). Measured
-// on the HunyuanVideo-shaped layer: 1 in 4 made the kernel slower (28.2 ->
-// 33.5 ms): the softmax is bound by its per-tile critical path, not by MUFU.
-constexpr int kPairEmuEvery = 0;
-[[maybe_unused]] constexpr int kEmuMod = kPairEmuEvery > 0 ? kPairEmuEvery : 1;
 constexpr int kPairLaunchRegs = 168;   // per thread at launch (3 warps per sub-partition)
 constexpr int kPairSoftmaxRegs = 224;  // softmax warpgroups after setmaxnreg.inc
 constexpr int kPairOtherRegs = 56;     // producer / MMA warpgroup after setmaxnreg.dec
@@ -777,25 +772,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const float alpha = rebase ? fast_exp2(m - m_new) : 1.0f;  // exp2(-inf) = 0
       const float m_use = m_new == -INFINITY ? 0.0f : m_new;
       float s0 = 0.0f, s1 = 0.0f;
-      // Full tiles may evaluate one pair in kPairEmuEvery on the FMA pipe; the
-      // ragged tile uses MUFU only.
-      [[maybe_unused]] const bool full_tile = kvalid == BK;
 #pragma unroll
       for (int ch = 0; ch < BK / 32; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c0 = ch * 32 + 2 * i;
-          float y0, y1, e0, e1;
+          float y0, y1;
           ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -m_use, -m_use);
-          bool emulate = false;
-          if constexpr (kPairEmuEvery > 0) emulate = full_tile && i % kEmuMod == kEmuMod - 1;
-          if (emulate) {
-            exp2_poly2(e0, e1, y0, y1);
-          } else {
-            e0 = fast_exp2(y0);
-            e1 = fast_exp2(y1);
-          }
+          const float e0 = fast_exp2(y0);
+          const float e1 = fast_exp2(y1);
           fadd2(s0, s1, s0, s1, e0, e1);
           pk[i] = pack_bf16x2(e0, e1);
         }

@@ -82,6 +82,10 @@ MaskGeom make_mask_geom(const Dims& d, int32_t kind);
 
 // Device address of this module's status word on the current device.
 int* device_status_word(cudaError_t* err);
+// Identity of the calling thread's current CUDA context, or NULL when none is
+// current yet (the runtime makes the device's primary context current on its
+// first call that needs one).
+void* current_context();
 
 // Tensor map of a [BH, N, d] bf16 tensor with a (64 x rows x 1) box, 128-byte swizzle.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int32_t d, int32_t N, int32_t BH,

@@ -868,21 +868,26 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / 
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_scratch_mutex;
 float* g_scratch_ptr[kMaxScratchDevices] = {};
+void* g_scratch_ctx[kMaxScratchDevices] = {};  // context the cached address belongs to
 
 // Device address of the current device's copy of g_noalloc_scratch. In host
 // code the array's name is only a stand-in, so the address is looked up with
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress with that device current: on the first call on each
+// device, and again whenever the device's context changed since (after a
+// cudaDeviceReset the module is loaded again, at another address).
 cudaError_t noalloc_scratch(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (g_scratch_ptr[dev] == nullptr || ctx == nullptr || g_scratch_ctx[dev] != ctx) {
     void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);  // initialises the context if needed
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = static_cast<float*>(ptr);
+    g_scratch_ctx[dev] = current_context();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;

@@ -9,8 +9,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "exp2_poly_coeffs.h"
-
 namespace svg {
 
 // Device-side error bits, OR-ed into a per-module status word.
@@ -310,29 +308,6 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
   asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
-}
-
-// 2^y0, 2^y1 on the FMA/ALU pipes instead of the MUFU unit: y = n + f with
-// n = round(y) (adding and removing 1.5*2^23 rounds to an integer in fp32) and
-// f in [-1/2, 1/2]; 2^f by the minimax cubic of exp2_poly_coeffs.h; 2^n by
-// adding n to the exponent field (the integer bits of y + 1.5*2^23 shifted
-// left by 23 are exactly n << 23). Inputs are clamped to >= -125 so every
-// result stays a normal number (below that the result is some value in
-// (0, 2^-124], negligible next to a softmax row maximum >= 1); the kernels
-// only pass finite y <= 2^8.
-__device__ __forceinline__ void exp2_poly2(float& r0, float& r1, float y0, float y1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  y0 = fmaxf(y0, -125.0f);
-  y1 = fmaxf(y1, -125.0f);
-  float t0, t1, n0, n1, f0, f1, p0, p1;
-  fadd2(t0, t1, y0, y1, kShift, kShift);
-  fadd2(n0, n1, t0, t1, -kShift, -kShift);
-  fadd2(f0, f1, y0, y1, -n0, -n1);
-  ffma2(p0, p1, f0, f1, kExp2Poly3, kExp2Poly3, kExp2Poly2, kExp2Poly2);
-  ffma2(p0, p1, p0, p1, f0, f1, kExp2Poly1, kExp2Poly1);
-  ffma2(p0, p1, p0, p1, f0, f1, kExp2Poly0, kExp2Poly0);
-  r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Sets bits [a, b) (clipped to [0, 64)) of a 64-bit set held in 2 words.
