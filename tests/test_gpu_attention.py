@@ -151,15 +151,20 @@ def test_empty_csr_rows_give_zero(svg):
     status_clean()
 
 
-FULL = [SI.COGVIDEOX, SI.HUNYUAN, SI.LONG] + SI.sweep_workloads()
+# planted inputs for every workload, plus unstructured ones (Q, K, V ~ N(0, 1):
+# diffuse attention, every computed block matters) at the two model shapes
+FULL = [(w, True) for w in [SI.COGVIDEOX, SI.HUNYUAN, SI.LONG] + SI.sweep_workloads()] + \
+    [(SI.COGVIDEOX, False), (SI.HUNYUAN, False)]
 
 
-@pytest.mark.parametrize("wl", FULL, ids=lambda w: w.name)
-def test_sparse_attention_full_size_sampled_rows(svg, wl):
+@pytest.mark.parametrize("wl,planted", FULL,
+                         ids=lambda x: x if not isinstance(x, bool) else
+                         ("planted" if x else "unstructured"))
+def test_sparse_attention_full_size_sampled_rows(svg, wl, planted):
     """The full workload through the same launch as the benchmark; the oracle
     checks sampled rows (edges + random) of a few heads of each label."""
     g = svg.Geom.from_workload(wl)
-    q, k, v = SI.make_qkv(wl)
+    q, k, v = SI.make_qkv(wl, planted=planted)
     kinds = SI.planted_head_kinds(wl)
     labels = torch.tensor(kinds * wl.B, dtype=torch.int8)
     layer = _layer(svg, g, n_samples=wl.n_samples)
@@ -180,5 +185,7 @@ def test_sparse_attention_full_size_sampled_rows(svg, wl):
             qn, kn, vn = to_f64(q[b, h]), to_f64(k[b, h]), to_f64(v[b, h])
             want, _ = O.layer_rows(qn, kn, vn, kinds[h], wl.T, wl.P, wl.n_text, wl.spatial_band,
                                    wl.temporal_width, wl.block_q, wl.block_k, wl.scale, rows=rows)
-            assert_close(to_f64(o[b, h, torch.from_numpy(rows)]), want, f"{wl.name} b{b} h{h}")
+            assert_close(to_f64(o[b, h, torch.from_numpy(rows)]), want,
+                         f"{wl.name} {'planted' if planted else 'unstructured'} b{b} h{h} "
+                         f"label {kinds[h]}")
     status_clean()

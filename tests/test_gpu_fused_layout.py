@@ -99,17 +99,20 @@ def test_fused_equals_explicit_bitwise_and_oracle(svg, case, labels_kind, layout
     status_clean()
 
 
-FULL = [(SI.COGVIDEOX, "fused"), (SI.HUNYUAN, "fused"), (SI.LONG, "fused"),
-        (SI.sweep_workloads()[4], "fused"), (SI.HUNYUAN, "gathered")]
+FULL = [(SI.COGVIDEOX, "fused", True), (SI.HUNYUAN, "fused", True), (SI.LONG, "fused", True),
+        (SI.sweep_workloads()[4], "fused", True), (SI.HUNYUAN, "gathered", True),
+        (SI.HUNYUAN, "fused", False)]
 
 
-@pytest.mark.parametrize("wl,layout", FULL, ids=lambda x: x if isinstance(x, str) else x.name)
-def test_fused_full_size(svg, wl, layout):
+@pytest.mark.parametrize("wl,layout,planted", FULL,
+                         ids=lambda x: x if isinstance(x, str) else
+                         (("planted" if x else "unstructured") if isinstance(x, bool) else x.name))
+def test_fused_full_size(svg, wl, layout, planted):
     """The benchmark's workloads: fused == explicit bit for bit over every
     output element, and sampled rows of a few heads of each label against the
-    oracle."""
+    oracle (planted inputs, and unstructured N(0, 1) ones)."""
     g = svg.Geom.from_workload(wl)
-    q, k, v = SI.make_qkv(wl)
+    q, k, v = SI.make_qkv(wl, planted=planted)
     kinds = SI.planted_head_kinds(wl)
     labels = torch.tensor(kinds * wl.B, dtype=torch.int8)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
