@@ -359,6 +359,52 @@ def layer_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, label: int, T: int, 
     return sparse_attention_rows(qp, kp, vp, bm, block_q, block_k, scale, layout_rows)
 
 
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) quantisation of V for the FP8 PV product
+# ---------------------------------------------------------------------------
+# The project article "Sparse-VideoGen and the sparsity hiding inside video
+# diffusion attention" (section "Publication record and the road ahead") lists
+# FP8 attention as an open item; the pages fix no format or scheme. The one
+# checked here: E4M3 in its "fn" form (1 sign, 4 exponent bits with bias 7, 3
+# mantissa bits, no infinities, largest finite value 448 = 1.75 * 2^8, smallest
+# normal 2^-6, subnormal spacing 2^-9), values rounded to nearest with ties to
+# even and saturated to +-448; one scale per (head, channel).
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest E4M3 value of each x (ties to even), saturating to +-448.
+
+    In a binade [2^e, 2^(e+1)) with e >= -6 the grid spacing is 2^(e-3); below
+    2^-6 (subnormals) it is 2^-9. Returns float64 values on the E4M3 grid."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    spacing = np.where(a >= 2.0 ** -6, 2.0 ** (e - 3), 2.0 ** -9)
+    q = np.round(a / spacing) * spacing  # numpy rounds halves to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.where(x < 0, -q, q)
+
+
+def quantize_v_e4m3(v: np.ndarray):
+    """Per-channel e4m3 quantisation of one head's V [N, d] (exact bf16 values).
+
+    amax_c = max_j |v_jc|; the code of v_jc is e4m3_round of the fp32 product
+    v_jc * fp32(448 / amax_c) (both the quotient and the product rounded to
+    fp32, the precision in which the rounding decision is taken); the scale is
+    fp32(amax_c / 448). A zero channel gets scale 0 and codes 0. Returns
+    (codes float64 [N, d] on the E4M3 grid, scale float32 [d]); v ~= codes * scale.
+    """
+    v32 = np.asarray(v, dtype=np.float32)
+    amax = np.max(np.abs(v32), axis=0).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, np.float32(E4M3_MAX) / amax, np.float32(0.0)).astype(np.float32)
+    x = (v32 * inv[None, :]).astype(np.float32)
+    codes = e4m3_round(x.astype(np.float64))
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    return codes, scale
+
+
 def flops_computed_blocks(bm: np.ndarray, N: int, block_q: int, block_k: int, d: int) -> int:
     """Algorithmic FLOPs of block-sparse attention: 4*d per computed (row, key) pair."""
     rows_in = np.minimum(block_q, N - np.arange(bm.shape[0]) * block_q)
