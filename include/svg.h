@@ -274,6 +274,203 @@ svg_status svg_sparse_attention_fused(const svg_geom* geom, const svg_bf16* q,
                                       svg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * svg_quantize_v_e4m3 -- V for the FP8 PV product of
+ * svg_sparse_attention_fp8pv. The project article "Sparse-VideoGen and the
+ * sparsity hiding inside video diffusion attention" (section "Publication
+ * record and the road ahead") lists FP8 attention as open; the pages fix no
+ * scheme, so this one is stated here. One scale per (b, h, channel):
+ *   amax_c     = max over the head's N rows of |v[b,h,j,c]|,
+ *   v8[b,h,j,c] = e4m3(v[b,h,j,c] * (448 / amax_c))  (fp32 product, round to
+ *                nearest even, saturating; E4M3 "fn": bias 7, max 448),
+ *   v_scale[b,h,c] = amax_c / 448, so v ~= v8 * v_scale
+ * (an all-zero channel gets scale 0 and codes 0). Each head is read in the
+ * layout it attends in: from v (frame-major) when labelled spatial or when
+ * labels is NULL, from vp (position-major) when labelled temporal.
+ *   v, vp      device bf16 [B,H,N,128]; vp may be NULL when labels is NULL.
+ *   labels     device int8 [B*H] or NULL.
+ *   v8         device uint8 [B,H,N,128] out (e4m3 codes), 16-byte aligned.
+ *   v_scale    device float [B*H*128] out.
+ * Errors: INVALID_ARG, UNSUPPORTED (head_dim != 128), CUDA.
+ */
+svg_status svg_quantize_v_e4m3(const svg_geom* geom, const svg_bf16* v, const svg_bf16* vp,
+                               const int8_t* labels, uint8_t* v8, float* v_scale,
+                               svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * svg_sparse_attention_fp8pv -- svg_sparse_attention with the PV product in
+ * FP8 (tcgen05 kind::f8f6f4): the softmax probabilities are rounded to e4m3
+ * (scaled by 2^6, which the row sum carries too, so it cancels) and multiplied
+ * with the e4m3 V of svg_quantize_v_e4m3; the fp32 accumulator is scaled back
+ * per channel by v_scale before the division by the row sum. Q K^T, the
+ * softmax and the output stay as in svg_sparse_attention, so the result is the
+ * same block-sparse attention up to e4m3 rounding of P and V (unit roundoff
+ * 2^-4 each): a looser tolerance than the bf16 product's.
+ *   q, k, qp, kp, labels, CSR, o, op, lse   as for svg_sparse_attention
+ *                  (qp, kp, op NULL together when no head is temporal).
+ *   v8, v_scale    from svg_quantize_v_e4m3 with the same labels (every head
+ *                  in its own layout).
+ * Errors: INVALID_ARG, UNSUPPORTED (head_dim != 128, block_q != 128, or a
+ *   device where the paired-tile kernel cannot run), CUDA.
+ */
+svg_status svg_sparse_attention_fp8pv(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                                      const svg_bf16* qp, const svg_bf16* kp, const uint8_t* v8,
+                                      const float* v_scale, const int8_t* labels,
+                                      const int32_t* row_ptr_s, const int32_t* col_idx_s,
+                                      const int32_t* row_ptr_t, const int32_t* col_idx_t,
+                                      svg_bf16* o, svg_bf16* op, float* lse,
+                                      svg_stream_t stream);
+
+/* ===========================================================================
+ * Semantic-aware permutation (Sparse VideoGen 2)
+ * The project article "Sparse-VideoGen and the sparsity hiding inside video
+ * diffusion attention", section "Three generations of the same idea": the
+ * second generation clusters tokens by meaning (a batched, "flash" k-means),
+ * permutes them so each cluster is contiguous, and runs a dynamic block-sparse
+ * attention over the permuted layout; the install section names block sparse
+ * attention with varied block sizes. The pages give no formula; the rules of
+ * each call below are stated with it. Every tensor is per (b, h) = bh, heads
+ * stacked: x [BH, N, d] bf16, centroids [BH, C, d] fp32, assign/order
+ * [BH, N] int32, offsets [BH, C+1] int32. All device memory is the caller's.
+ * ------------------------------------------------------------------------ */
+
+/* svg2_kmeans_workspace_bytes -- host only: device workspace (256-byte
+ * aligned) svg2_kmeans and svg2_kmeans_step need. Errors: INVALID_ARG,
+ * UNSUPPORTED (d not 64/128; C not a multiple of 16 in [16, 256]). */
+svg_status svg2_kmeans_workspace_bytes(int32_t BH, int32_t N, int32_t d, int32_t C,
+                                       size_t* bytes);
+
+/* svg2_kmeans -- Lloyd's k-means of every head's N rows of x (the query or the
+ * key vectors of a layer) into C clusters, `iters` iterations:
+ *   init        centroid c = row floor(c * N / C) of the head;
+ *   assignment  every row to the centroid of least squared Euclidean distance,
+ *               the centroids rounded to bf16 for the distance (a tcgen05
+ *               product X C^T, fp32 accumulation), ties to the smaller index;
+ *   update      each centroid = the fp32 mean of its members, summed in sorted
+ *               order (an empty cluster keeps its centroid).
+ * Outputs the final centroids, the last iteration's assignment (the one the
+ * centroids are the means of) and its stable cluster order: order[bh, pos] =
+ * row at sorted position pos (rows sorted by cluster, ties by row index),
+ * offsets[bh, c] = first sorted position of cluster c, offsets[bh, C] = N.
+ * With iters = 0: the initial centroids, their assignment and its order.
+ * Deterministic (fixed-order sums, integer atomics only).
+ * Errors: INVALID_ARG (null, misaligned: x and centroids 16-byte, workspace
+ * 256-byte), UNSUPPORTED (d, C), CAPACITY (workspace), CUDA. */
+svg_status svg2_kmeans(int32_t BH, int32_t N, int32_t d, int32_t C, int32_t iters,
+                       const svg_bf16* x, float* centroids, int32_t* assign, int32_t* order,
+                       int32_t* offsets, void* workspace, size_t workspace_bytes,
+                       svg_stream_t stream);
+
+/* svg2_kmeans_step -- one iteration of svg2_kmeans from given centroids:
+ * assignment with centroids_in, its stable cluster order and offsets, and
+ * centroids_out = the members' means (centroids_in for empty clusters).
+ * centroids_out must not be centroids_in. Errors: as svg2_kmeans. */
+svg_status svg2_kmeans_step(int32_t BH, int32_t N, int32_t d, int32_t C, const svg_bf16* x,
+                            const float* centroids_in, float* centroids_out, int32_t* assign,
+                            int32_t* order, int32_t* offsets, void* workspace,
+                            size_t workspace_bytes, svg_stream_t stream);
+
+/* svg2_select_clusters -- the key clusters each query cluster attends. For
+ * query cluster a of head bh, key cluster b weighs
+ *   w_b = softmax_b( scale * cq[bh,a] . ck[bh,b] + log |b| ),  |b| =
+ *   offsets_k[bh,b+1] - offsets_k[bh,b]  (empty clusters weigh 0),
+ * and a keeps the fewest clusters, taken in descending weight (ties to the
+ * smaller index), whose weights add up to at least top_p (0 < top_p <= 1).
+ * With disp != NULL (SVG-EAR's error-aware routing; the project article's
+ * section "Three generations of the same idea": high-error blocks are computed
+ * exactly, the rest compensated), a skipped cluster is kept as well when its
+ * error estimate w_b * disp[bh, b] exceeds tau (disp from
+ * svg2_cluster_value_stats: the spread of what its centroid would stand in for).
+ *   cq [BH, Cq, d], ck [BH, Ck, d] fp32 centroids; offsets_k [BH, Ck+1].
+ *   disp  fp32 [BH, Ck] or NULL; tau >= 0 (ignored when disp is NULL).
+ *   sel   out, uint32 [BH, Cq, ceil(Ck/32)]: bit b%32 of word b/32 = kept.
+ * fp32 arithmetic; a cluster whose preceding weight lies within rounding of
+ * top_p (or whose estimate lies within rounding of tau) may go either way.
+ * Errors: INVALID_ARG (Ck > 1024, bad scale/top_p/tau), CUDA. */
+svg_status svg2_select_clusters(int32_t BH, int32_t d, int32_t Cq, int32_t Ck, float scale,
+                                float top_p, const float* cq, const float* ck,
+                                const int32_t* offsets_k, const float* disp, float tau,
+                                uint32_t* sel, svg_stream_t stream);
+
+/* svg2_cluster_value_stats -- SVG-EAR statistics of every key cluster, over
+ * its members in sorted order: vbar[bh, b] = the fp32 mean of their values,
+ * disp[bh, b] = sqrt(mean over members and channels of (v - vbar)^2); an
+ * empty cluster gets zeros. v bf16 [BH, N, d] (original order), order_k and
+ * offsets_k from svg2_kmeans of the keys; vbar fp32 [BH, Ck, d] (16-byte
+ * aligned), disp fp32 [BH, Ck]. Errors: INVALID_ARG, UNSUPPORTED (d), CUDA. */
+svg_status svg2_cluster_value_stats(int32_t BH, int32_t N, int32_t d, int32_t Ck,
+                                    const svg_bf16* v, const int32_t* order_k,
+                                    const int32_t* offsets_k, float* vbar, float* disp,
+                                    svg_stream_t stream);
+
+/* svg2_ear_workspace_bytes -- host only: the workspace of svg2_ear_compensate
+ * (bf16 copies of the centroids and value means). */
+svg_status svg2_ear_workspace_bytes(int32_t BH, int32_t d, int32_t Ck, size_t* bytes);
+
+/* svg2_ear_compensate -- SVG-EAR's centroid compensation ("parameter-free
+ * centroid compensation" of the skipped blocks, the same section), in place
+ * on the block-sparse output of svg2_sparse_attention. For sorted query row i
+ * of query tile r of head bh: every key outside the computed key tiles of row
+ * r of the CSR is stood in for by its cluster: n_b(r) uncovered keys of key
+ * cluster b add n_b(r) * exp(scale * q_i . kbar_b) to the softmax's
+ * denominator and the same times vbar_b to its numerator (kbar_b, vbar_b
+ * rounded to bf16, the tensor-core operand format), so
+ *   O_i = (O_s,i e^{lse_i} + sum_b n_b e^{scale q_i.kbar_b} vbar_b)
+ *         / (e^{lse_i} + sum_b n_b e^{scale q_i.kbar_b}).
+ *   qs         bf16 [BH, N, d] sorted queries (as given to the attention).
+ *   kbar       fp32 [BH, Ck, d] key centroids (svg2_kmeans of the keys).
+ *   vbar       fp32 [BH, Ck, d] (svg2_cluster_value_stats).
+ *   offsets_k  [BH, Ck+1]; row_ptr, col_idx the CSR the attention used
+ *              (block_q = 128, block_k).
+ *   os         bf16 [BH, N, d] in: the attention's output, out: compensated.
+ *   lse        fp32 [BH, N], the attention's log-sum-exp (natural log).
+ *   workspace  >= svg2_ear_workspace_bytes, 256-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED (d, block_k, Ck not a multiple of 16 in
+ * [16, 256], more than 4096 key tiles), CAPACITY, CUDA. */
+svg_status svg2_ear_compensate(int32_t BH, int32_t N, int32_t d, int32_t Ck, int32_t block_k,
+                               float scale, const svg_bf16* qs, const float* kbar,
+                               const float* vbar, const int32_t* offsets_k,
+                               const int32_t* row_ptr, const int32_t* col_idx, svg_bf16* os,
+                               const float* lse, void* workspace, size_t workspace_bytes,
+                               svg_stream_t stream);
+
+/* svg2_build_tile_csr -- the tile pairs of the sorted layouts to compute, one
+ * CSR per head: query tile r (sorted query positions [r*block_q, ...)) lists,
+ * ascending, every key tile holding a key of a cluster kept (sel) by a query
+ * cluster present in tile r. Row bh*nQB + r of the stacked CSR; row_ptr
+ * [BH*nQB + 1] (row_ptr[0] = 0), col_idx [col_capacity] (at most
+ * BH*nQB*nKB entries are written; beyond col_capacity an entry is dropped
+ * and the device bounds bit set). counts [BH*nQB] int32 is scratch.
+ * Errors: INVALID_ARG, UNSUPPORTED (blocks not 64/128, more than 4096 key
+ * tiles), CUDA. */
+svg_status svg2_build_tile_csr(int32_t BH, int32_t N, int32_t Cq, int32_t Ck, int32_t block_q,
+                               int32_t block_k, const int32_t* offsets_q, const int32_t* offsets_k,
+                               const uint32_t* sel, int32_t* row_ptr, int32_t* col_idx,
+                               int64_t col_capacity, int32_t* counts, svg_stream_t stream);
+
+/* svg2_gather_rows / svg2_scatter_rows -- the token permutation:
+ *   gather   y[bh, pos]            = x[bh, order[bh, pos]]   (into sorted order)
+ *   scatter  y[bh, order[bh, pos]] = y_sorted[bh, pos]       (back)
+ * x, y bf16 [BH, N, d] (d 64 or 128), 16-byte aligned, not overlapping. An
+ * order entry outside [0, N) sets the device bounds bit and is skipped. */
+svg_status svg2_gather_rows(int32_t BH, int32_t N, int32_t d, const svg_bf16* x,
+                            const int32_t* order, svg_bf16* y, svg_stream_t stream);
+svg_status svg2_scatter_rows(int32_t BH, int32_t N, int32_t d, const svg_bf16* y_sorted,
+                             const int32_t* order, svg_bf16* y, svg_stream_t stream);
+
+/* svg2_sparse_attention -- block-sparse flash attention over the sorted
+ * layouts with one CSR per head (from svg2_build_tile_csr with block_q =
+ * 128): for sorted query row i of head bh,
+ *   O[i] = sum over keys j of listed tiles of softmax_j(scale * q_i . k_j) v_j
+ * (queries sorted by their cluster order, keys and values by theirs; the same
+ * kernel as svg_sparse_attention). qs, ks, vs, os bf16 [BH, N, d]; lse fp32
+ * [BH, N] (natural log, sorted query rows) or NULL.
+ * Errors: INVALID_ARG, UNSUPPORTED (d or block_k), CUDA. */
+svg_status svg2_sparse_attention(int32_t BH, int32_t N, int32_t d, int32_t block_k, float scale,
+                                 const svg_bf16* qs, const svg_bf16* ks, const svg_bf16* vs,
+                                 const int32_t* row_ptr, const int32_t* col_idx, svg_bf16* os,
+                                 float* lse, svg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * svg_get_device_status -- synchronises `stream`, then reads and clears the
  * device status bits of the current device (1 = a bounded wait ran out,
  * 2 = an out-of-range index from caller memory was skipped) into *bits

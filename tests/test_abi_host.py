@@ -27,7 +27,7 @@ def svg():
 
 def _header_symbols():
     text = open(os.path.join(ROOT, "include", "svg.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:svg_status|const char\*|int32_t)\s+(svg_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:svg_status|const char\*|int32_t)\s+(svg2?_\w+)\s*\(",
                                  text, flags=re.M)))
 
 

@@ -35,7 +35,11 @@ STATUS_NAMES = {0: "SVG_OK", 1: "SVG_ERR_INVALID_ARG", 2: "SVG_ERR_UNSUPPORTED",
 EXPORTED = [
     "svg_mask_nnz", "svg_build_block_mask", "svg_profile_workspace_bytes",
     "svg_profile_heads", "svg_profile_heads_noalloc", "svg_permute", "svg_unpermute", "svg_permute_qkv",
-    "svg_sparse_attention", "svg_sparse_attention_fused", "svg_get_device_status", "svg_selftest_wait_timeout",
+    "svg_sparse_attention", "svg_sparse_attention_fused", "svg_quantize_v_e4m3",
+    "svg_sparse_attention_fp8pv", "svg_get_device_status", "svg_selftest_wait_timeout",
+    "svg2_kmeans_workspace_bytes", "svg2_kmeans", "svg2_kmeans_step", "svg2_select_clusters",
+    "svg2_build_tile_csr", "svg2_gather_rows", "svg2_scatter_rows", "svg2_sparse_attention",
+    "svg2_cluster_value_stats", "svg2_ear_workspace_bytes", "svg2_ear_compensate",
     "svg_status_string", "svg_version",
 ]
 
@@ -101,8 +105,22 @@ def load() -> ctypes.CDLL:
         "svg_permute_qkv": [_c_geom_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
         "svg_sparse_attention": [_c_geom_p] + [_vp] * 15,
         "svg_sparse_attention_fused": [_c_geom_p] + [_vp] * 13,
+        "svg_quantize_v_e4m3": [_c_geom_p] + [_vp] * 6,
+        "svg_sparse_attention_fp8pv": [_c_geom_p] + [_vp] * 15,
         "svg_get_device_status": [_vp, ctypes.POINTER(_i32)],
         "svg_selftest_wait_timeout": [_i64, _vp],
+        "svg2_kmeans_workspace_bytes": [_i32, _i32, _i32, _i32, ctypes.POINTER(_sz)],
+        "svg2_kmeans": [_i32, _i32, _i32, _i32, _i32] + [_vp] * 6 + [_sz, _vp],
+        "svg2_kmeans_step": [_i32, _i32, _i32, _i32] + [_vp] * 7 + [_sz, _vp],
+        "svg2_select_clusters": [_i32, _i32, _i32, _i32, ctypes.c_float, ctypes.c_float] +
+                                [_vp] * 4 + [ctypes.c_float, _vp, _vp],
+        "svg2_cluster_value_stats": [_i32] * 4 + [_vp] * 6,
+        "svg2_ear_workspace_bytes": [_i32, _i32, _i32, ctypes.POINTER(_sz)],
+        "svg2_ear_compensate": [_i32] * 5 + [ctypes.c_float] + [_vp] * 9 + [_sz, _vp],
+        "svg2_build_tile_csr": [_i32] * 6 + [_vp] * 5 + [_i64, _vp, _vp],
+        "svg2_gather_rows": [_i32, _i32, _i32, _vp, _vp, _vp, _vp],
+        "svg2_scatter_rows": [_i32, _i32, _i32, _vp, _vp, _vp, _vp],
+        "svg2_sparse_attention": [_i32, _i32, _i32, _i32, ctypes.c_float] + [_vp] * 8,
         "svg_status_string": [_i32],
         "svg_version": [],
     }
@@ -224,6 +242,21 @@ def svg_sparse_attention_fused(geom: Geom, q, k, v, kp, vp, labels, row_ptr_s, c
         _stream(stream)))
 
 
+def svg_quantize_v_e4m3(geom: Geom, v, vp, labels, v8, v_scale, stream=None) -> None:
+    _check("svg_quantize_v_e4m3", load().svg_quantize_v_e4m3(
+        ctypes.byref(geom), _ptr(v), _ptr(vp), _ptr(labels), _ptr(v8), _ptr(v_scale),
+        _stream(stream)))
+
+
+def svg_sparse_attention_fp8pv(geom: Geom, q, k, qp, kp, v8, v_scale, labels, row_ptr_s,
+                               col_idx_s, row_ptr_t, col_idx_t, o, op, lse=None,
+                               stream=None) -> None:
+    _check("svg_sparse_attention_fp8pv", load().svg_sparse_attention_fp8pv(
+        ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(qp), _ptr(kp), _ptr(v8), _ptr(v_scale),
+        _ptr(labels), _ptr(row_ptr_s), _ptr(col_idx_s), _ptr(row_ptr_t), _ptr(col_idx_t),
+        _ptr(o), _ptr(op), _ptr(lse), _stream(stream)))
+
+
 def svg_get_device_status(stream=None):
     """(status, bits): synchronises the stream and reads/clears the device status bits."""
     bits = _i32(0)
@@ -234,3 +267,85 @@ def svg_get_device_status(stream=None):
 def svg_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
     _check("svg_selftest_wait_timeout",
            load().svg_selftest_wait_timeout(limit_cycles, _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# semantic-aware permutation (Sparse VideoGen 2)
+# ---------------------------------------------------------------------------
+def svg2_kmeans_workspace_bytes(BH: int, N: int, d: int, C: int) -> int:
+    out = _sz(0)
+    _check("svg2_kmeans_workspace_bytes",
+           load().svg2_kmeans_workspace_bytes(BH, N, d, C, ctypes.byref(out)))
+    return out.value
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def svg2_kmeans(BH, N, d, C, iters, x, centroids, assign, order, offsets, workspace,
+                stream=None) -> None:
+    _check("svg2_kmeans", load().svg2_kmeans(
+        BH, N, d, C, iters, _ptr(x), _ptr(centroids), _ptr(assign), _ptr(order), _ptr(offsets),
+        _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def svg2_kmeans_step(BH, N, d, C, x, centroids_in, centroids_out, assign, order, offsets,
+                     workspace, stream=None) -> None:
+    _check("svg2_kmeans_step", load().svg2_kmeans_step(
+        BH, N, d, C, _ptr(x), _ptr(centroids_in), _ptr(centroids_out), _ptr(assign), _ptr(order),
+        _ptr(offsets), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def svg2_select_clusters(BH, d, Cq, Ck, scale, top_p, cq, ck, offsets_k, sel, disp=None,
+                         tau=0.0, stream=None) -> None:
+    _check("svg2_select_clusters", load().svg2_select_clusters(
+        BH, d, Cq, Ck, scale, top_p, _ptr(cq), _ptr(ck), _ptr(offsets_k), _ptr(disp), tau,
+        _ptr(sel), _stream(stream)))
+
+
+def svg2_cluster_value_stats(BH, N, d, Ck, v, order_k, offsets_k, vbar, disp,
+                             stream=None) -> None:
+    _check("svg2_cluster_value_stats", load().svg2_cluster_value_stats(
+        BH, N, d, Ck, _ptr(v), _ptr(order_k), _ptr(offsets_k), _ptr(vbar), _ptr(disp),
+        _stream(stream)))
+
+
+def svg2_ear_workspace_bytes(BH, d, Ck) -> int:
+    out = _sz(0)
+    _check("svg2_ear_workspace_bytes", load().svg2_ear_workspace_bytes(BH, d, Ck,
+                                                                       ctypes.byref(out)))
+    return out.value
+
+
+def svg2_ear_compensate(BH, N, d, Ck, block_k, scale, qs, kbar, vbar, offsets_k, row_ptr,
+                        col_idx, os, lse, workspace, stream=None) -> None:
+    _check("svg2_ear_compensate", load().svg2_ear_compensate(
+        BH, N, d, Ck, block_k, scale, _ptr(qs), _ptr(kbar), _ptr(vbar), _ptr(offsets_k),
+        _ptr(row_ptr), _ptr(col_idx), _ptr(os), _ptr(lse), _ptr(workspace), _nbytes(workspace),
+        _stream(stream)))
+
+
+def svg2_build_tile_csr(BH, N, Cq, Ck, block_q, block_k, offsets_q, offsets_k, sel, row_ptr,
+                        col_idx, counts, col_capacity=None, stream=None) -> None:
+    cap = col_idx.numel() if col_capacity is None else col_capacity
+    _check("svg2_build_tile_csr", load().svg2_build_tile_csr(
+        BH, N, Cq, Ck, block_q, block_k, _ptr(offsets_q), _ptr(offsets_k), _ptr(sel),
+        _ptr(row_ptr), _ptr(col_idx), cap, _ptr(counts), _stream(stream)))
+
+
+def svg2_gather_rows(BH, N, d, x, order, y, stream=None) -> None:
+    _check("svg2_gather_rows", load().svg2_gather_rows(BH, N, d, _ptr(x), _ptr(order), _ptr(y),
+                                                       _stream(stream)))
+
+
+def svg2_scatter_rows(BH, N, d, y_sorted, order, y, stream=None) -> None:
+    _check("svg2_scatter_rows", load().svg2_scatter_rows(BH, N, d, _ptr(y_sorted), _ptr(order),
+                                                         _ptr(y), _stream(stream)))
+
+
+def svg2_sparse_attention(BH, N, d, block_k, scale, qs, ks, vs, row_ptr, col_idx, os,
+                          lse=None, stream=None) -> None:
+    _check("svg2_sparse_attention", load().svg2_sparse_attention(
+        BH, N, d, block_k, scale, _ptr(qs), _ptr(ks), _ptr(vs), _ptr(row_ptr), _ptr(col_idx),
+        _ptr(os), _ptr(lse), _stream(stream)))

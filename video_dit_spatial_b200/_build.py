@@ -14,7 +14,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsvg.so")
 
-SOURCES = ["api.cu", "permute.cu", "block_mask.cu", "profile.cu", "attention.cu"]
+SOURCES = ["api.cu", "permute.cu", "block_mask.cu", "profile.cu", "attention.cu", "quant.cu", "svg2.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",

@@ -33,8 +33,12 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
+// Driver entry points are looked up under a mutex of their own, which is never
+// held while anything else is called.
+std::mutex g_entry_mutex;
+
 EncodeTiledFn encode_fn() {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::mutex> lock(g_entry_mutex);
   if (g_encode == nullptr) {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -47,7 +51,7 @@ EncodeTiledFn encode_fn() {
 }
 
 CtxGetCurrentFn ctx_get_fn() {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::mutex> lock(g_entry_mutex);
   if (g_ctx_get == nullptr) {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -145,17 +149,22 @@ int* device_status_word(cudaError_t* err) {
     *err = cudaErrorInvalidDevice;
     return nullptr;
   }
-  void* ctx = current_context();
-  std::lock_guard<std::mutex> lock(g_mutex);
   // A device reset tears the context down and the module is loaded again into
-  // the next one, at a new address: look it up again whenever the context changes.
-  if (g_status_ptr[dev] == nullptr || ctx == nullptr || g_status_ctx[dev] != ctx) {
-    void* ptr = nullptr;
-    *err = cudaGetSymbolAddress(&ptr, g_device_status);  // initialises the context if needed
-    if (*err != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(ptr);
-    g_status_ctx[dev] = current_context();
+  // the next one, at a new address: look it up again whenever the context
+  // changes. No lock is held while the runtime or the driver is called.
+  void* ctx = current_context();
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_status_ptr[dev] != nullptr && ctx != nullptr && g_status_ctx[dev] == ctx)
+      return g_status_ptr[dev];
   }
+  void* ptr = nullptr;
+  *err = cudaGetSymbolAddress(&ptr, g_device_status);  // initialises the context if needed
+  if (*err != cudaSuccess) return nullptr;
+  void* now = current_context();
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_status_ptr[dev] = static_cast<int*>(ptr);
+  g_status_ctx[dev] = now;
   return g_status_ptr[dev];
 }
 
@@ -170,6 +179,21 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int32_t d, int32_t N, in
   const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_u8_rows128(CUtensorMap* map, const void* base, int32_t N, int32_t BH,
+                          int32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {128u, 128u * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -370,11 +394,64 @@ svg_status svg_sparse_attention(const svg_geom* geom, const svg_bf16* q, const s
   int* status = svg::device_status_word(&err);
   if (status == nullptr) return SVG_ERR_CUDA;
   svg::AttnArgs a{q, k, v, qp, kp, vp, labels, row_ptr_s, col_idx_s, row_ptr_t, col_idx_t,
-                  o, op, lse, false};
+                  o, op, lse, false, nullptr, nullptr};
   if (svg::launch_sparse_attention(d, a, status, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return SVG_ERR_CUDA;
   return SVG_OK;
+}
+
+svg_status svg_quantize_v_e4m3(const svg_geom* geom, const svg_bf16* v, const svg_bf16* vp,
+                               const int8_t* labels, uint8_t* v8, float* v_scale,
+                               svg_stream_t stream) {
+  if (v == nullptr || v8 == nullptr || v_scale == nullptr) return SVG_ERR_INVALID_ARG;
+  if (labels != nullptr && vp == nullptr) return SVG_ERR_INVALID_ARG;
+  if (!svg::aligned16(v) || !svg::aligned16(v8) || (vp != nullptr && !svg::aligned16(vp)) ||
+      (reinterpret_cast<uintptr_t>(v_scale) & 3u) != 0)
+    return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_geom(geom, false);
+  if (st != SVG_OK) return st;
+  if (geom->head_dim != 128) return SVG_ERR_UNSUPPORTED;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  return svg::launch_quantize_v(d, v, vp, labels, v8, v_scale,
+                                static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVG_OK
+             : SVG_ERR_CUDA;
+}
+
+svg_status svg_sparse_attention_fp8pv(const svg_geom* geom, const svg_bf16* q, const svg_bf16* k,
+                                      const svg_bf16* qp, const svg_bf16* kp, const uint8_t* v8,
+                                      const float* v_scale, const int8_t* labels,
+                                      const int32_t* row_ptr_s, const int32_t* col_idx_s,
+                                      const int32_t* row_ptr_t, const int32_t* col_idx_t,
+                                      svg_bf16* o, svg_bf16* op, float* lse,
+                                      svg_stream_t stream) {
+  if (q == nullptr || k == nullptr || v8 == nullptr || v_scale == nullptr || o == nullptr ||
+      row_ptr_s == nullptr || col_idx_s == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  const bool any_perm = qp || kp || op;
+  const bool all_perm = qp && kp && op;
+  if (any_perm && !all_perm) return SVG_ERR_INVALID_ARG;
+  if (all_perm && (row_ptr_t == nullptr || col_idx_t == nullptr)) return SVG_ERR_INVALID_ARG;
+  const void* tensors[6] = {q, k, o, qp, kp, op};
+  for (int t = 0; t < 6; ++t)
+    if (tensors[t] != nullptr && !svg::aligned16(tensors[t])) return SVG_ERR_INVALID_ARG;
+  if (!svg::aligned16(v8) || (reinterpret_cast<uintptr_t>(v_scale) & 3u) != 0)
+    return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_geom(geom, true);
+  if (st != SVG_OK) return st;
+  if (geom->head_dim != 128 || geom->block_q != 128) return SVG_ERR_UNSUPPORTED;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  const Dims d = svg::make_dims(*geom);
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  svg::AttnArgs a{q, k, nullptr, qp, kp, nullptr, labels, row_ptr_s, col_idx_s, row_ptr_t,
+                  col_idx_t, o, op, lse, false, v8, v_scale};
+  err = svg::launch_sparse_attention(d, a, status, static_cast<cudaStream_t>(stream));
+  if (err == cudaErrorNotSupported) return SVG_ERR_UNSUPPORTED;
+  return err == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
 }
 
 svg_status svg_sparse_attention_fused(const svg_geom* geom, const svg_bf16* q,
@@ -405,8 +482,245 @@ svg_status svg_sparse_attention_fused(const svg_geom* geom, const svg_bf16* q,
   int* status = svg::device_status_word(&err);
   if (status == nullptr) return SVG_ERR_CUDA;
   svg::AttnArgs a{q, k, v, nullptr, kp, vp, labels, row_ptr_s, col_idx_s,
-                  row_ptr_t, col_idx_t, o, nullptr, lse, true};
+                  row_ptr_t, col_idx_t, o, nullptr, lse, true, nullptr, nullptr};
   err = svg::launch_sparse_attention(d, a, status, static_cast<cudaStream_t>(stream));
+  if (err == cudaErrorNotSupported) return SVG_ERR_UNSUPPORTED;
+  return err == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// semantic-aware permutation (Sparse VideoGen 2)
+// ---------------------------------------------------------------------------
+static svg_status check_kmeans_shape(int32_t BH, int32_t N, int32_t d, int32_t C) {
+  if (BH < 1 || BH > 65535 || N < 1 || N > (1 << 30)) return SVG_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  if (C < 16 || C > 256 || C % 16 != 0) return SVG_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(BH) * N > 0x7fffffffLL) return SVG_ERR_INVALID_ARG;
+  return SVG_OK;
+}
+
+svg_status svg2_kmeans_workspace_bytes(int32_t BH, int32_t N, int32_t d, int32_t C,
+                                       size_t* bytes) {
+  if (bytes == nullptr) return SVG_ERR_INVALID_ARG;
+  const svg_status st = check_kmeans_shape(BH, N, d, C);
+  if (st != SVG_OK) return st;
+  *bytes = svg::kmeans_workspace_bytes(BH, N, d, C);
+  return SVG_OK;
+}
+
+static svg_status kmeans_common(int32_t BH, int32_t N, int32_t d, int32_t C, const svg_bf16* x,
+                                const float* c_in, float* c_out, int32_t* assign, int32_t* order,
+                                int32_t* offsets, void* ws, size_t ws_bytes, int** status) {
+  if (x == nullptr || c_out == nullptr || assign == nullptr || order == nullptr ||
+      offsets == nullptr || ws == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  svg_status st = check_kmeans_shape(BH, N, d, C);
+  if (st != SVG_OK) return st;
+  if (!svg::aligned16(x) || !svg::aligned16(c_out) || (c_in && !svg::aligned16(c_in)) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(assign) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(order) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(offsets) & 3u) != 0)
+    return SVG_ERR_INVALID_ARG;
+  if (ws_bytes < svg::kmeans_workspace_bytes(BH, N, d, C)) return SVG_ERR_CAPACITY;
+  if ((st = svg::check_device()) != SVG_OK) return st;
+  cudaError_t err;
+  *status = svg::device_status_word(&err);
+  return *status == nullptr ? SVG_ERR_CUDA : SVG_OK;
+}
+
+svg_status svg2_kmeans(int32_t BH, int32_t N, int32_t d, int32_t C, int32_t iters,
+                       const svg_bf16* x, float* centroids, int32_t* assign, int32_t* order,
+                       int32_t* offsets, void* workspace, size_t workspace_bytes,
+                       svg_stream_t stream) {
+  if (iters < 0 || iters > 1000) return SVG_ERR_INVALID_ARG;
+  int* status = nullptr;
+  const svg_status st = kmeans_common(BH, N, d, C, x, nullptr, centroids, assign, order, offsets,
+                                      workspace, workspace_bytes, &status);
+  if (st != SVG_OK) return st;
+  return svg::launch_kmeans(BH, N, d, C, iters, x, centroids, assign, order, offsets, workspace,
+                            status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVG_OK
+             : SVG_ERR_CUDA;
+}
+
+svg_status svg2_kmeans_step(int32_t BH, int32_t N, int32_t d, int32_t C, const svg_bf16* x,
+                            const float* centroids_in, float* centroids_out, int32_t* assign,
+                            int32_t* order, int32_t* offsets, void* workspace,
+                            size_t workspace_bytes, svg_stream_t stream) {
+  if (centroids_in == nullptr || centroids_in == centroids_out) return SVG_ERR_INVALID_ARG;
+  int* status = nullptr;
+  const svg_status st = kmeans_common(BH, N, d, C, x, centroids_in, centroids_out, assign, order,
+                                      offsets, workspace, workspace_bytes, &status);
+  if (st != SVG_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (svg::launch_kmeans_assign(BH, N, d, C, x, centroids_in, assign, workspace, status, s) !=
+          cudaSuccess ||
+      svg::launch_cluster_sort(BH, N, C, assign, order, offsets, workspace, d, status, s) !=
+          cudaSuccess ||
+      svg::launch_kmeans_update(BH, N, d, C, x, order, offsets, centroids_in, centroids_out, s) !=
+          cudaSuccess)
+    return SVG_ERR_CUDA;
+  return SVG_OK;
+}
+
+svg_status svg2_select_clusters(int32_t BH, int32_t d, int32_t Cq, int32_t Ck, float scale,
+                                float top_p, const float* cq, const float* ck,
+                                const int32_t* offsets_k, const float* disp, float tau,
+                                uint32_t* sel, svg_stream_t stream) {
+  if (cq == nullptr || ck == nullptr || offsets_k == nullptr || sel == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  if (BH < 1 || BH > 65535 || d < 1 || d > 4096 || Cq < 1 || Cq > 65535 || Ck < 1 || Ck > 1024)
+    return SVG_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !(scale < 3.0e38f) || !(top_p > 0.0f) || !(top_p <= 1.0f))
+    return SVG_ERR_INVALID_ARG;
+  if (disp != nullptr && !(tau >= 0.0f)) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  return svg::launch_select_clusters(BH, d, Cq, Ck, scale, top_p, cq, ck, offsets_k, disp, tau,
+                                     sel, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVG_OK
+             : SVG_ERR_CUDA;
+}
+
+svg_status svg2_cluster_value_stats(int32_t BH, int32_t N, int32_t d, int32_t Ck,
+                                    const svg_bf16* v, const int32_t* order_k,
+                                    const int32_t* offsets_k, float* vbar, float* disp,
+                                    svg_stream_t stream) {
+  if (v == nullptr || order_k == nullptr || offsets_k == nullptr || vbar == nullptr ||
+      disp == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  if (BH < 1 || BH > 65535 || N < 1 || Ck < 1 || static_cast<int64_t>(BH) * N > 0x7fffffffLL)
+    return SVG_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  if (!svg::aligned16(v) || (reinterpret_cast<uintptr_t>(vbar) & 15u) != 0)
+    return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  return svg::launch_cluster_stats(BH, N, d, Ck, v, order_k, offsets_k, vbar, disp,
+                                   static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVG_OK
+             : SVG_ERR_CUDA;
+}
+
+svg_status svg2_ear_workspace_bytes(int32_t BH, int32_t d, int32_t Ck, size_t* bytes) {
+  if (bytes == nullptr || BH < 1 || Ck < 1) return SVG_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  *bytes = svg::ear_workspace_bytes(BH, d, Ck);
+  return SVG_OK;
+}
+
+svg_status svg2_ear_compensate(int32_t BH, int32_t N, int32_t d, int32_t Ck, int32_t block_k,
+                               float scale, const svg_bf16* qs, const float* kbar,
+                               const float* vbar, const int32_t* offsets_k,
+                               const int32_t* row_ptr, const int32_t* col_idx, svg_bf16* os,
+                               const float* lse, void* workspace, size_t workspace_bytes,
+                               svg_stream_t stream) {
+  if (qs == nullptr || kbar == nullptr || vbar == nullptr || offsets_k == nullptr ||
+      row_ptr == nullptr || col_idx == nullptr || os == nullptr || lse == nullptr ||
+      workspace == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  if (BH < 1 || BH > 65535 || N < 1 || N > (1 << 30)) return SVG_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  if (Ck < 16 || Ck > 256 || Ck % 16 != 0) return SVG_ERR_UNSUPPORTED;
+  if (block_k != 64 && block_k != 128) return SVG_ERR_UNSUPPORTED;
+  if ((N + block_k - 1) / block_k > 4096) return SVG_ERR_UNSUPPORTED;
+  if (!(scale > 0.0f) || !(scale < 3.0e38f)) return SVG_ERR_INVALID_ARG;
+  if (!svg::aligned16(qs) || !svg::aligned16(os) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SVG_ERR_INVALID_ARG;
+  if (workspace_bytes < svg::ear_workspace_bytes(BH, d, Ck)) return SVG_ERR_CAPACITY;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  return svg::launch_ear_compensate(BH, N, d, Ck, block_k, scale, qs, kbar, vbar, offsets_k,
+                                    row_ptr, col_idx, os, lse, workspace, status,
+                                    static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVG_OK
+             : SVG_ERR_CUDA;
+}
+
+svg_status svg2_build_tile_csr(int32_t BH, int32_t N, int32_t Cq, int32_t Ck, int32_t block_q,
+                               int32_t block_k, const int32_t* offsets_q, const int32_t* offsets_k,
+                               const uint32_t* sel, int32_t* row_ptr, int32_t* col_idx,
+                               int64_t col_capacity, int32_t* counts, svg_stream_t stream) {
+  if (offsets_q == nullptr || offsets_k == nullptr || sel == nullptr || row_ptr == nullptr ||
+      col_idx == nullptr || counts == nullptr || col_capacity < 0)
+    return SVG_ERR_INVALID_ARG;
+  if (BH < 1 || BH > 65535 || N < 1 || N > (1 << 30) || Cq < 1 || Ck < 1 || Ck > 1024)
+    return SVG_ERR_INVALID_ARG;
+  if ((block_q != 64 && block_q != 128) || (block_k != 64 && block_k != 128))
+    return SVG_ERR_UNSUPPORTED;
+  const int64_t nqb = (N + block_q - 1) / block_q, nkb = (N + block_k - 1) / block_k;
+  if (nkb > 4096) return SVG_ERR_UNSUPPORTED;
+  if (BH * nqb > 0x7fffffffLL / 2) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  return svg::launch_tile_csr(BH, N, Cq, Ck, block_q, block_k, offsets_q, offsets_k, sel, row_ptr,
+                              col_idx, col_capacity, counts, status,
+                              static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVG_OK
+             : SVG_ERR_CUDA;
+}
+
+static svg_status rows_common(int32_t BH, int32_t N, int32_t d, const svg_bf16* x,
+                              const int32_t* order, svg_bf16* y, bool scatter,
+                              svg_stream_t stream) {
+  if (x == nullptr || order == nullptr || y == nullptr) return SVG_ERR_INVALID_ARG;
+  if (BH < 1 || N < 1 || static_cast<int64_t>(BH) * N > 0x7fffffffLL) return SVG_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SVG_ERR_UNSUPPORTED;
+  if (!svg::aligned16(x) || !svg::aligned16(y)) return SVG_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(BH) * N * d * 2;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(x), b0 = reinterpret_cast<uintptr_t>(y);
+  if (a0 < b0 + bytes && b0 < a0 + bytes) return SVG_ERR_INVALID_ARG;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  return svg::launch_permute_rows(BH, N, d, x, order, y, scatter, status,
+                                  static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVG_OK
+             : SVG_ERR_CUDA;
+}
+
+svg_status svg2_gather_rows(int32_t BH, int32_t N, int32_t d, const svg_bf16* x,
+                            const int32_t* order, svg_bf16* y, svg_stream_t stream) {
+  return rows_common(BH, N, d, x, order, y, false, stream);
+}
+
+svg_status svg2_scatter_rows(int32_t BH, int32_t N, int32_t d, const svg_bf16* y_sorted,
+                             const int32_t* order, svg_bf16* y, svg_stream_t stream) {
+  return rows_common(BH, N, d, y_sorted, order, y, true, stream);
+}
+
+svg_status svg2_sparse_attention(int32_t BH, int32_t N, int32_t d, int32_t block_k, float scale,
+                                 const svg_bf16* qs, const svg_bf16* ks, const svg_bf16* vs,
+                                 const int32_t* row_ptr, const int32_t* col_idx, svg_bf16* os,
+                                 float* lse, svg_stream_t stream) {
+  if (qs == nullptr || ks == nullptr || vs == nullptr || row_ptr == nullptr ||
+      col_idx == nullptr || os == nullptr)
+    return SVG_ERR_INVALID_ARG;
+  if (!svg::aligned16(qs) || !svg::aligned16(ks) || !svg::aligned16(vs) || !svg::aligned16(os))
+    return SVG_ERR_INVALID_ARG;
+  if (BH < 1 || BH > 65535 || N < 1 || N > (1 << 30)) return SVG_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !(scale < 3.0e38f)) return SVG_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || (block_k != 64 && block_k != 128)) return SVG_ERR_UNSUPPORTED;
+  svg_status st = svg::check_device();
+  if (st != SVG_OK) return st;
+  // the sorted layouts are one sequence of N tokens per head, no text part
+  svg_geom g{1, BH, 1, N, 0, d, 128, block_k, 0, 0, scale};
+  const Dims dm = svg::make_dims(g);
+  cudaError_t err;
+  int* status = svg::device_status_word(&err);
+  if (status == nullptr) return SVG_ERR_CUDA;
+  svg::AttnArgs a{qs, ks, vs, nullptr, nullptr, nullptr, nullptr, row_ptr, col_idx, nullptr,
+                  nullptr, os, nullptr, lse, false, nullptr, nullptr, true};
+  err = svg::launch_sparse_attention(dm, a, status, static_cast<cudaStream_t>(stream));
   if (err == cudaErrorNotSupported) return SVG_ERR_UNSUPPORTED;
   return err == cudaSuccess ? SVG_OK : SVG_ERR_CUDA;
 }

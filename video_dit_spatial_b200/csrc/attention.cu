@@ -67,6 +67,10 @@ struct Cfg {
 // likewise with `gather_kv`, else tiled maps over position-major copies.
 struct __align__(64) AttnParams {
   CUtensorMap tm_q[2], tm_k[2], tm_v[2];  // [0]: frame-major, [1]: position-major
+  // FP8 PV: e4m3 V of every head in its own layout (one 8-bit tiled map) and
+  // the per-(head, channel) scales that undo its quantisation
+  CUtensorMap tm_v8;
+  const float* v_scale;
   const int8_t* labels;
   const int32_t* row_ptr[2];
   const int32_t* col_idx[2];
@@ -75,6 +79,7 @@ struct __align__(64) AttnParams {
   int* status;
   int32_t N, Nv, BH, nqb, nkb, bq, bk;
   int32_t has_permuted;
+  int32_t csr_per_head;  // CSR row of (bh, query block r) is bh * nqb + r
   int32_t gather, gather_kv, T, P;
   float scale_log2;
 };
@@ -121,8 +126,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) atomicOr(p.status, kDevErrBounds);
     return;
   }
-  const int32_t rp0 = __ldg(p.row_ptr[sel] + qb);
-  int32_t n = __ldg(p.row_ptr[sel] + qb + 1) - rp0;
+  const int csr_row = (p.csr_per_head ? bh * p.nqb : 0) + qb;
+  const int32_t rp0 = __ldg(p.row_ptr[sel] + csr_row);
+  int32_t n = __ldg(p.row_ptr[sel] + csr_row + 1) - rp0;
   if (n < 0 || n > p.nkb) {
     if (tid == 0) atomicOr(p.status, kDevErrBounds);
     n = 0;
@@ -397,6 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // S_t(j) also retires PV_t(j-1) (the softmax may then re-base O_t freely).
 // ===========================================================================
 constexpr int kPairThreads = 384;
+constexpr float kRebaseLog2F8 = 2.0f;  // FP8 PV: lazy re-basing threshold (log2 units)
+constexpr float kPShiftLog2F8 = 6.0f;  // FP8 PV: P is scaled by 2^6 before rounding
 constexpr int kPairProducerWarp = 8;
 constexpr int kPairMmaWarp = 9;
 constexpr int kPairLaunchRegs = 168;   // per thread at launch (3 warps per sub-partition)
@@ -414,18 +422,21 @@ struct PairBarriers {
   int abort_flag;
 };
 
-template <int D, int BK>
+template <int D, int BK, bool F8 = false>
 struct PairCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kQPanel = 128 * 128;
   static constexpr int kKVPanel = BK * 128;
   static constexpr int kQBytes = kPanels * kQPanel;     // one query tile
-  static constexpr int kKVBytes = kPanels * kKVPanel;   // one K (or V) tile
-  static constexpr int kStages = (D == 128 && BK == 128) ? 2 : 3;
+  static constexpr int kKVBytes = kPanels * kKVPanel;   // one K (or bf16 V) tile
+  // FP8 PV: a V tile is BK rows of D = 128 e4m3 bytes, one 128-byte swizzled panel
+  static constexpr int kVBytes = F8 ? BK * 128 : kKVBytes;
+  static constexpr int kKStages = (D == 128 && BK == 128) ? 2 : 3;
+  static constexpr int kVStages = F8 ? 3 : kKStages;
   static constexpr int kOffQ = 0;                        // Q_A, then Q_B
   static constexpr int kOffK = kOffQ + 2 * kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kVBytes;
   static constexpr int kBarBytes = (static_cast<int>(sizeof(PairBarriers)) + 127) / 128 * 128;
   static constexpr int kUsed = kOffBar + kBarBytes + 1024;
   static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
@@ -435,6 +446,9 @@ struct PairCfg {
   static __device__ __forceinline__ uint32_t col_o(int t) { return t ? 384u : 128u; }
   static_assert(kOffBar + kBarBytes + 1024 <= kSmem, "bookkeeping must fit the allocation");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+  static_assert(kKStages <= 3 && kVStages <= 3, "ring barriers hold 3 stages");
+  static_assert(!F8 || D == 128, "FP8 PV takes 128-byte e4m3 rows (d = 128)");
+  static_assert(kVBytes % 1024 == 0 && kKVBytes % 1024 == 0, "swizzled tiles stay 1024-aligned");
 };
 
 
@@ -455,10 +469,16 @@ struct UnionWalk {
   }
 };
 
-template <int D, int BK>
+// F8: the PV product in FP8 (kind::f8f6f4): P rounded to e4m3 (scaled by 2^6
+// through the exponent, with the lazy re-basing threshold lowered to 2^2 so P
+// stays below 2^8 < 448 and mostly above e4m3's subnormal range) times V in
+// e4m3 with one scale per (head, channel); QK^T stays bf16.
+template <int D, int BK, bool F8 = false>
 __global__ void __launch_bounds__(kPairThreads, 1)
     sparse_attention_pair_kernel(const __grid_constant__ AttnParams p) {
-  using C = PairCfg<D, BK>;
+  using C = PairCfg<D, BK, F8>;
+  constexpr float kRebase = F8 ? kRebaseLog2F8 : kRebaseLog2;
+  constexpr float kPShift = F8 ? kPShiftLog2F8 : 0.0f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -509,8 +529,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     nt[t] = 0;
     cols[t] = p.col_idx[sel];
     if (qb[t] < p.nqb) {
-      const int32_t r0 = __ldg(p.row_ptr[sel] + qb[t]);
-      int32_t len = __ldg(p.row_ptr[sel] + qb[t] + 1) - r0;
+      const int csr_row = (p.csr_per_head ? bh * p.nqb : 0) + qb[t];
+      const int32_t r0 = __ldg(p.row_ptr[sel] + csr_row);
+      int32_t len = __ldg(p.row_ptr[sel] + csr_row + 1) - r0;
       if (len < 0 || len > p.nkb) {
         if (tid == 0) atomicOr(p.status, kDevErrBounds);
         len = 0;
@@ -527,9 +548,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   }
   if (tid == 32) {
     mbar_init(&bar->q_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
     }
@@ -597,34 +620,37 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           int c = walk.next(ia, ib);
           if (!ia && !ib) break;
           if (c < 0 || c >= p.nkb) c = 0;  // flagged and masked by the softmax warps
-          const int st = u % C::kStages;
-          const uint32_t par = ((u / C::kStages) & 1) ^ 1;
+          const int sk = u % C::kKStages;
+          const int sv = u % C::kVStages;
           bool ok = true;
           if (lane == 0) {
-            ok = mbar_wait(&bar->k_empty[st], par, abort_flag, p.status);
-            if (ok) mbar_arrive_expect_tx(&bar->k_full[st], C::kKVBytes);
+            ok = mbar_wait(&bar->k_empty[sk], ((u / C::kKStages) & 1) ^ 1, abort_flag, p.status);
+            if (ok) mbar_arrive_expect_tx(&bar->k_full[sk], C::kKVBytes);
           }
           if (!__shfl_sync(0xffffffffu, ok, 0)) break;
           if (gather_kv) {
-            gather_rows(sK + st * C::kKVBytes, mk, &bar->k_full[st], c * BK, BK, C::kKVPanel, keep);
+            gather_rows(sK + sk * C::kKVBytes, mk, &bar->k_full[sk], c * BK, BK, C::kKVPanel, keep);
           } else if (lane == 0) {
             for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_load_3d_hint(sK + st * C::kKVBytes + pn * C::kKVPanel, mk, &bar->k_full[st],
+              tma_load_3d_hint(sK + sk * C::kKVBytes + pn * C::kKVPanel, mk, &bar->k_full[sk],
                                pn * 64, c * BK, bh, keep);
           }
           if (lane == 0) {
-            ok = mbar_wait(&bar->v_empty[st], par, abort_flag, p.status);
-            if (ok) mbar_arrive_expect_tx(&bar->v_full[st], C::kKVBytes);
+            ok = mbar_wait(&bar->v_empty[sv], ((u / C::kVStages) & 1) ^ 1, abort_flag, p.status);
+            if (ok) mbar_arrive_expect_tx(&bar->v_full[sv], C::kVBytes);
           }
           if (!__shfl_sync(0xffffffffu, ok, 0)) {
             issued = -(u + 1);  // K of step u is in flight, V is not
             break;
           }
-          if (gather_kv) {
-            gather_rows(sV + st * C::kKVBytes, mv, &bar->v_full[st], c * BK, BK, C::kKVPanel, keep);
+          if constexpr (F8) {
+            if (lane == 0)
+              tma_load_3d_hint(sV + sv * C::kVBytes, &p.tm_v8, &bar->v_full[sv], 0, c * BK, bh, keep);
+          } else if (gather_kv) {
+            gather_rows(sV + sv * C::kVBytes, mv, &bar->v_full[sv], c * BK, BK, C::kKVPanel, keep);
           } else if (lane == 0) {
             for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_load_3d_hint(sV + st * C::kKVBytes + pn * C::kKVPanel, mv, &bar->v_full[st],
+              tma_load_3d_hint(sV + sv * C::kVBytes + pn * C::kKVPanel, mv, &bar->v_full[sv],
                                pn * 64, c * BK, bh, keep);
           }
           issued = u + 1;
@@ -632,13 +658,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (lane == 0 && *abort_flag) {
           // Let every copy this warp started land before the CTA retires.
           const int done = issued < 0 ? -issued : issued;
-          for (int u = (done > C::kStages ? done - C::kStages : 0); u < done; ++u) {
-            const int st = u % C::kStages;
-            const uint32_t par = (u / C::kStages) & 1;
-            const bool v_issued = issued >= 0 || u < done - 1;
+          for (int u = (done > C::kKStages ? done - C::kKStages : 0); u < done; ++u) {
             long long t0 = clock64();
-            while (!(mbar_try_wait(&bar->k_full[st], par) &&
-                     (!v_issued || mbar_try_wait(&bar->v_full[st], par))) &&
+            while (!mbar_try_wait(&bar->k_full[u % C::kKStages], (u / C::kKStages) & 1) &&
+                   clock64() - t0 < kWaitLimitCycles) {
+            }
+          }
+          const int v_done = issued >= 0 ? done : done - 1;
+          for (int u = (v_done > C::kVStages ? v_done - C::kVStages : 0); u < v_done; ++u) {
+            long long t0 = clock64();
+            while (!mbar_try_wait(&bar->v_full[u % C::kVStages], (u / C::kVStages) & 1) &&
                    clock64() - t0 < kWaitLimitCycles) {
             }
           }
@@ -648,7 +677,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // ------------------------------------------------------------ MMA issuer
       if (lane_id() == 0 && any_work) {
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BK, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        constexpr uint32_t idesc_pv =
+            F8 ? idesc_e4m3_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
         const uint32_t q_addr = smem_u32(sQ);
         const uint32_t k_addr = smem_u32(sK);
         const uint32_t v_addr = smem_u32(sV);
@@ -662,31 +692,43 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           walk.next(in[0], in[1]);
           const bool step = in[0] || in[1];  // false: drain step after the last block
           if (!step && !prev_in[0] && !prev_in[1]) break;
-          const int st = u % C::kStages;
-          const int pst = (u + C::kStages - 1) % C::kStages;
+          const int st = u % C::kKStages;
+          const int pst = (u + C::kVStages - 1) % C::kVStages;
           bool k_ready = false, v_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (prev_in[t]) {  // PV_t of the previous step
               if (!v_ready) {
-                ok = mbar_wait(&bar->v_full[pst], ((u - 1) / C::kStages) & 1, abort_flag, p.status);
+                ok = mbar_wait(&bar->v_full[pst], ((u - 1) / C::kVStages) & 1, abort_flag, p.status);
                 v_ready = true;
               }
               if (ok) ok = mbar_wait(&bar->p_full[t], pv_done[t] & 1, abort_flag, p.status);
               if (!ok) break;
               tc_fence_after();
+              if constexpr (F8) {
+                // K = 32 keys per MMA: 8 tensor-memory columns of four e4m3 P values,
+                // 32 rows of 128 e4m3 V bytes (one 128-byte swizzle atom across d)
   #pragma unroll
-              for (int kk = 0; kk < BK / 16; ++kk) {
-                const uint64_t b = sdesc_sw128(v_addr + pst * C::kKVBytes + kk * 16 * 128,
-                                               C::kKVPanel, 1024);
-                mma_bf16_ts(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv,
+                for (int kk = 0; kk < BK / 32; ++kk) {
+                  const uint64_t b = sdesc_sw128(v_addr + pst * C::kVBytes + kk * 32 * 128,
+                                                 C::kVBytes, 1024);
+                  mma_f8_ts(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv,
                             (pv_done[t] > 0 || kk > 0) ? 1u : 0u);
+                }
+              } else {
+  #pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                  const uint64_t b = sdesc_sw128(v_addr + pst * C::kVBytes + kk * 16 * 128,
+                                                 C::kKVPanel, 1024);
+                  mma_bf16_ts(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv,
+                              (pv_done[t] > 0 || kk > 0) ? 1u : 0u);
+                }
               }
               ++pv_done[t];
               if (pv_done[t] == nt[t]) tc_commit(&bar->o_final[t]);
             }
             if (step && in[t]) {  // QK_t of this step
               if (!k_ready) {
-                ok = mbar_wait(&bar->k_full[st], (u / C::kStages) & 1, abort_flag, p.status);
+                ok = mbar_wait(&bar->k_full[st], (u / C::kKStages) & 1, abort_flag, p.status);
                 k_ready = true;
                 if (!ok) break;
               }
@@ -767,25 +809,44 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const float m_tile =
           fmaxf(fmax3(xm[0], xm[1], xm[2]), fmax3(xm[3], fmax3(xm[4], xm[5], xm[6]), xm[7])) *
           p.scale_log2;
-      const bool rebase = m_tile > m + kRebaseLog2;
+      const bool rebase = m_tile > m + kRebase;
       const float m_new = rebase ? m_tile : m;
       const float alpha = rebase ? fast_exp2(m - m_new) : 1.0f;  // exp2(-inf) = 0
-      const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+      // FP8: the probabilities (and so the row sum) carry a factor 2^kPShift
+      const float m_use = (m_new == -INFINITY ? 0.0f : m_new) - kPShift;
       float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll
       for (int ch = 0; ch < BK / 32; ++ch) {
-        uint32_t pk[16];
+        if constexpr (F8) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = ch * 32 + 2 * i;
-          float y0, y1;
-          ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -m_use, -m_use);
-          const float e0 = fast_exp2(y0);
-          const float e1 = fast_exp2(y1);
-          fadd2(s0, s1, s0, s1, e0, e1);
-          pk[i] = pack_bf16x2(e0, e1);
+          for (int i = 0; i < 8; ++i) {
+            const int c0 = ch * 32 + 4 * i;
+            float y0, y1, y2, y3;
+            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -m_use, -m_use);
+            ffma2(y2, y3, u2f(sr[c0 + 2]), u2f(sr[c0 + 3]), p.scale_log2, p.scale_log2, -m_use,
+                  -m_use);
+            const float e0 = fast_exp2(y0), e1 = fast_exp2(y1);
+            const float e2 = fast_exp2(y2), e3 = fast_exp2(y3);
+            fadd2(s0, s1, s0, s1, e0, e1);
+            fadd2(s0, s1, s0, s1, e2, e3);
+            pk[i] = pack_e4m3x4(e0, e1, e2, e3);
+          }
+          tmem_st_32x32b_x8(s_col + ch * 8, pk);
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = ch * 32 + 2 * i;
+            float y0, y1;
+            ffma2(y0, y1, u2f(sr[c0]), u2f(sr[c0 + 1]), p.scale_log2, p.scale_log2, -m_use, -m_use);
+            const float e0 = fast_exp2(y0);
+            const float e1 = fast_exp2(y1);
+            fadd2(s0, s1, s0, s1, e0, e1);
+            pk[i] = pack_bf16x2(e0, e1);
+          }
+          tmem_st_32x32b_x16(s_col + ch * 16, pk);
         }
-        tmem_st_32x32b_x16(s_col + ch * 16, pk);
       }
       l = l * alpha + (s0 + s1);
       m = m_new;
@@ -824,6 +885,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tmem_ld_wait();
         reg_fence(o);
       }
+      if constexpr (F8) {  // undo V's per-channel quantisation scale
+        const float* vs = p.v_scale + static_cast<size_t>(bh) * D + ch * 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * __ldg(vs + i));
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
@@ -837,7 +903,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     if (p.lse != nullptr && row_valid) {
       p.lse[static_cast<size_t>(bh) * p.N + out_row] =
-          (have_o && l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          (have_o && l > 0.0f) ? (m + __log2f(l) - kPShift) * 0.69314718055994531f : -INFINITY;
     }
   }
 
@@ -852,10 +918,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 template <int D, int BK>
 cudaError_t launch_impl(const Dims& d, const AttnParams& p, cudaStream_t stream);
 
-template <int D, int BK>
+template <int D, int BK, bool F8 = false>
 cudaError_t launch_pair(const Dims& d, const AttnParams& p, cudaStream_t stream) {
-  using C = PairCfg<D, BK>;
-  auto kern = sparse_attention_pair_kernel<D, BK>;
+  using C = PairCfg<D, BK, F8>;
+  auto kern = sparse_attention_pair_kernel<D, BK, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   // The register hand-over inside the kernel is only balanced when the kernel
@@ -868,8 +934,8 @@ cudaError_t launch_pair(const Dims& d, const AttnParams& p, cudaStream_t stream)
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kPairThreads, C::kSmem);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kPairLaunchRegs || resident < 1) {
-    // the single-tile kernel has no row gathers
-    if (p.gather) return cudaErrorNotSupported;
+    // the single-tile kernel has no row gathers and no FP8 product
+    if (p.gather || F8) return cudaErrorNotSupported;
     return launch_impl<D, BK>(d, p, stream);
   }
   dim3 grid(static_cast<unsigned>(((d.nqb + 1) / 2) * d.BH));
@@ -894,12 +960,20 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
                                     cudaStream_t stream) {
   AttnParams p;
   memset(&p, 0, sizeof(p));
+  const bool f8 = a.v8 != nullptr;
   const bool perm = a.qp != nullptr && !a.fused;
   if (a.fused && d.bq != 128) return cudaErrorNotSupported;
+  if (f8 && (d.bq != 128 || d.d != 128 || a.fused)) return cudaErrorNotSupported;
   if (!make_tmap_bf16(&p.tm_q[0], a.q, d.d, d.N, d.BH, d.bq) ||
-      !make_tmap_bf16(&p.tm_k[0], a.k, d.d, d.N, d.BH, d.bk) ||
-      !make_tmap_bf16(&p.tm_v[0], a.v, d.d, d.N, d.BH, d.bk))
+      !make_tmap_bf16(&p.tm_k[0], a.k, d.d, d.N, d.BH, d.bk))
     return cudaErrorInvalidValue;
+  if (f8) {
+    if (!make_tmap_u8_rows128(&p.tm_v8, a.v8, d.N, d.BH, d.bk)) return cudaErrorInvalidValue;
+    p.v_scale = a.v_scale;
+    p.tm_v[0] = p.tm_k[0];  // unused by the FP8 product
+  } else if (!make_tmap_bf16(&p.tm_v[0], a.v, d.d, d.N, d.BH, d.bk)) {
+    return cudaErrorInvalidValue;
+  }
   if (a.fused) {
     const int64_t rows = static_cast<int64_t>(d.BH) * d.N;
     if (!make_tmap_rows_bf16(&p.tm_q[1], a.q, d.d, rows)) return cudaErrorInvalidValue;
@@ -913,9 +987,13 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
     }
   } else if (perm) {
     if (!make_tmap_bf16(&p.tm_q[1], a.qp, d.d, d.N, d.BH, d.bq) ||
-        !make_tmap_bf16(&p.tm_k[1], a.kp, d.d, d.N, d.BH, d.bk) ||
-        !make_tmap_bf16(&p.tm_v[1], a.vp, d.d, d.N, d.BH, d.bk))
+        !make_tmap_bf16(&p.tm_k[1], a.kp, d.d, d.N, d.BH, d.bk))
       return cudaErrorInvalidValue;
+    if (f8) {
+      p.tm_v[1] = p.tm_k[1];  // unused by the FP8 product
+    } else if (!make_tmap_bf16(&p.tm_v[1], a.vp, d.d, d.N, d.BH, d.bk)) {
+      return cudaErrorInvalidValue;
+    }
   } else {
     p.tm_q[1] = p.tm_q[0];
     p.tm_k[1] = p.tm_k[0];
@@ -938,11 +1016,16 @@ cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* statu
   p.bq = d.bq;
   p.bk = d.bk;
   p.has_permuted = perm && a.op != nullptr && a.row_ptr_t != nullptr && a.col_idx_t != nullptr;
+  p.csr_per_head = a.csr_per_head ? 1 : 0;
   p.gather = a.fused ? 1 : 0;
   p.gather_kv = a.fused && a.kp == nullptr ? 1 : 0;
   p.T = d.T;
   p.P = d.P;
   p.scale_log2 = d.scale * 1.4426950408889634f;
+  if (f8) {
+    if (d.bk == 128) return launch_pair<128, 128, true>(d, p, stream);
+    return launch_pair<128, 64, true>(d, p, stream);
+  }
   if (d.bq == 128) {
     if (d.d == 128 && d.bk == 128) return launch_pair<128, 128>(d, p, stream);
     if (d.d == 128 && d.bk == 64) return launch_pair<128, 64>(d, p, stream);

@@ -90,6 +90,10 @@ void* current_context();
 // Tensor map of a [BH, N, d] bf16 tensor with a (64 x rows x 1) box, 128-byte swizzle.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int32_t d, int32_t N, int32_t BH,
                     int32_t box_rows);
+// Tensor map of a [BH, N, 128] 8-bit tensor with a (128 x rows x 1) box (one
+// 128-byte row per token), 128-byte swizzle.
+bool make_tmap_u8_rows128(CUtensorMap* map, const void* base, int32_t N, int32_t BH,
+                          int32_t box_rows);
 // Row map of the same tensor seen as [BH*N, d] with a 64 x 1 box, 128-byte
 // swizzle: the tensor map of tile::gather4 row gathers.
 bool make_tmap_rows_bf16(CUtensorMap* map, const void* base, int32_t d, int64_t rows);
@@ -108,6 +112,12 @@ struct AttnArgs {
   svg_bf16 *o, *op;
   float* lse;
   bool fused;  // temporal heads gather from q, k, v and scatter to o (qp..op unused)
+  // FP8 PV (v and vp unused): e4m3 V of every head in its own layout and the
+  // per-(head, channel) scales, as written by svg_quantize_v_e4m3
+  const uint8_t* v8;
+  const float* v_scale;
+  // one CSR per (b, h): row b*H*nQB + h*nQB + r, i.e. (bh * nQB + r)
+  bool csr_per_head = false;
 };
 cudaError_t launch_sparse_attention(const Dims& d, const AttnArgs& a, int* status,
                                     cudaStream_t stream);
@@ -130,6 +140,48 @@ cudaError_t launch_profile(const Dims& d, const ProfileArgs& a, int* status, cud
 size_t profile_noalloc_scratch_bytes();
 cudaError_t launch_profile_noalloc(const Dims& d, const ProfileArgs& a, int* status,
                                    cudaStream_t stream);
+
+// e4m3 quantisation of V (each head read from v or, if labelled temporal, vp):
+// amax per (head, channel) into v_scale, the codes into v8, then v_scale
+// turned into the dequantisation scale amax / 448.
+cudaError_t launch_quantize_v(const Dims& d, const svg_bf16* v, const svg_bf16* vp,
+                              const int8_t* labels, uint8_t* v8, float* v_scale,
+                              cudaStream_t stream);
+
+// Semantic-aware permutation (svg2.cu).
+size_t kmeans_workspace_bytes(int32_t BH, int32_t N, int32_t D, int32_t C);
+cudaError_t launch_kmeans(int32_t BH, int32_t N, int32_t D, int32_t C, int32_t iters,
+                          const svg_bf16* x, float* centroids, int32_t* assign, int32_t* order,
+                          int32_t* offsets, void* ws, int* status, cudaStream_t stream);
+cudaError_t launch_kmeans_assign(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
+                                 const float* centroids, int32_t* assign, void* ws, int* status,
+                                 cudaStream_t stream);
+cudaError_t launch_cluster_sort(int32_t BH, int32_t N, int32_t C, const int32_t* assign,
+                                int32_t* order, int32_t* offsets, void* ws, int32_t D, int* status,
+                                cudaStream_t stream);
+cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
+                                 const int32_t* order, const int32_t* offsets, const float* c_in,
+                                 float* c_out, cudaStream_t stream);
+cudaError_t launch_select_clusters(int32_t BH, int32_t D, int32_t Cq, int32_t Ck, float scale,
+                                   float top_p, const float* cq, const float* ck,
+                                   const int32_t* offsets_k, const float* disp, float tau,
+                                   uint32_t* sel, cudaStream_t stream);
+cudaError_t launch_cluster_stats(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* v,
+                                 const int32_t* order, const int32_t* offsets, float* vbar,
+                                 float* disp, cudaStream_t stream);
+size_t ear_workspace_bytes(int32_t BH, int32_t D, int32_t C);
+cudaError_t launch_ear_compensate(int32_t BH, int32_t N, int32_t D, int32_t C, int32_t bk,
+                                  float scale, const svg_bf16* qs, const float* kbar,
+                                  const float* vbar, const int32_t* offsets_k,
+                                  const int32_t* row_ptr, const int32_t* col_idx, svg_bf16* os,
+                                  const float* lse, void* ws, int* status, cudaStream_t stream);
+cudaError_t launch_tile_csr(int32_t BH, int32_t N, int32_t Cq, int32_t Ck, int32_t bq, int32_t bk,
+                            const int32_t* offsets_q, const int32_t* offsets_k, const uint32_t* sel,
+                            int32_t* row_ptr, int32_t* col_idx, int64_t capacity, int32_t* counts,
+                            int* status, cudaStream_t stream);
+cudaError_t launch_permute_rows(int32_t BH, int32_t N, int32_t D, const svg_bf16* x,
+                                const int32_t* order, svg_bf16* y, bool scatter, int* status,
+                                cudaStream_t stream);
 
 cudaError_t launch_wait_selftest(long long limit_cycles, int* status, cudaStream_t stream);
 

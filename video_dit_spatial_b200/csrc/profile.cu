@@ -880,15 +880,22 @@ cudaError_t noalloc_scratch(float** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  // No lock is held while the runtime or the driver is called.
   void* ctx = current_context();
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr || ctx == nullptr || g_scratch_ctx[dev] != ctx) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);  // initialises the context if needed
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = static_cast<float*>(ptr);
-    g_scratch_ctx[dev] = current_context();
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_ptr[dev] != nullptr && ctx != nullptr && g_scratch_ctx[dev] == ctx) {
+      *out = g_scratch_ptr[dev];
+      return cudaSuccess;
+    }
   }
+  void* ptr = nullptr;
+  e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);  // initialises the context if needed
+  if (e != cudaSuccess) return e;
+  void* now = current_context();
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  g_scratch_ptr[dev] = static_cast<float*>(ptr);
+  g_scratch_ctx[dev] = now;
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
 }

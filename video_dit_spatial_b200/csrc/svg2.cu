@@ -1,0 +1,1212 @@
+// Semantic-aware permutation (Sparse VideoGen 2). The project article
+// "Sparse-VideoGen and the sparsity hiding inside video diffusion attention",
+// section "Three generations of the same idea", describes the second
+// generation as semantic-aware sparse attention on an efficient token
+// permutation, run by a dynamic attention kernel and a flash (batched) k-means
+// kernel; the install section names block-sparse attention with varied block
+// sizes. The pages give no formula; the rules implemented here are:
+//   k-means     per (b, h), Lloyd iterations on the query (resp. key) vectors:
+//               initial centroids are the rows floor(c * N / C); each iteration
+//               assigns every row to its nearest centroid (squared Euclidean
+//               distance with the centroids rounded to bf16, ties to the
+//               smaller index) and replaces each centroid by the mean of its
+//               members (an empty cluster keeps its centroid);
+//   permutation tokens stably sorted by cluster, so each cluster is one run;
+//   selection   query cluster a keeps the fewest key clusters, in descending
+//               softmax_b(scale * c_q[a] . c_k[b] + log |b|) weight (ties to
+//               the smaller index), whose weights reach top_p;
+//   attention   block-granular on the sorted layouts: a (query tile, key tile)
+//               pair is computed iff a query cluster present in the query tile
+//               keeps a key cluster present in the key tile (the block-sparse
+//               attention kernel with one CSR per head).
+//
+// Kernels:
+//   kmeans_prep_kernel     fp32 centroids -> bf16 copy + squared norms
+//   kmeans_assign_kernel   tcgen05: S = X C^T for 128 rows x all C centroids
+//                          in tensor memory, then a per-row argmin of
+//                          |c|^2 - 2 x.c (one softmax-style warpgroup)
+//   sort_hist / sort_scan / sort_rank   stable counting sort by cluster
+//   kmeans_update_kernel   per cluster, the members' mean in sorted order
+//   select_kernel          the top-p key clusters of each query cluster
+//   tile_count / tile_fill kernels      per-head CSR of the tile pairs
+//   gather / scatter rows  the permutation of Q, K, V and of the output
+// All reductions run in a fixed order: results are deterministic.
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace svg {
+namespace {
+
+// ------------------------------------------------------------ assignment
+constexpr int kAsgThreads = 192;  // warps 0-3 argmin, 4 producer, 5 MMA
+constexpr int kAsgProducer = 4;
+constexpr int kAsgMma = 5;
+constexpr int kMaxC = 256;  // centroids per assignment launch (one MMA N)
+
+struct AsgBarriers {
+  uint64_t c_full;
+  uint64_t x_full[2], x_empty[2];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+struct AsgCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kXPanel = 128 * 128;      // 128 rows x 128 B
+  static constexpr int kXBytes = kPanels * kXPanel;
+  static constexpr int kCPanel = kMaxC * 128;    // up to 256 centroid rows x 128 B
+  static constexpr int kCBytes = kPanels * kCPanel;
+  static constexpr int kOffC = 0;
+  static constexpr int kOffX = kOffC + kCBytes;
+  static constexpr int kOffNorm = kOffX + 2 * kXBytes;
+  static constexpr int kOffBar = kOffNorm + kMaxC * 4;
+  static constexpr int kBarBytes = (static_cast<int>(sizeof(AsgBarriers)) + 127) / 128 * 128;
+  static constexpr int kUsed = kOffBar + kBarBytes + 1024;
+  // one CTA per SM: each takes all 512 tensor-memory columns
+  static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+  static_assert(kOffX % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles 1024-aligned");
+};
+
+struct __align__(64) AsgParams {
+  CUtensorMap tm_x;   // [BH, N, D] bf16, box (64, 128)
+  CUtensorMap tm_c;   // [BH, C, D] bf16, box (64, C)
+  const float* norms; // [BH, C]
+  int32_t* assign;    // [BH, N]
+  int* status;
+  int32_t N, C, n_tiles, ctas_per_head;
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+template <int D>
+__global__ void __launch_bounds__(kAsgThreads, 1)
+    kmeans_assign_kernel(const __grid_constant__ AsgParams p) {
+  using Cf = AsgCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sC = smem + Cf::kOffC;
+  uint8_t* sX = smem + Cf::kOffX;
+  float* sNorm = reinterpret_cast<float*>(smem + Cf::kOffNorm);
+  AsgBarriers* bar = reinterpret_cast<AsgBarriers*>(smem + Cf::kOffBar);
+  volatile int* abort_flag = &bar->abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int bh = blockIdx.y;
+  // this CTA's row tiles: [t0, t1)
+  const int t0 = static_cast<int>(static_cast<long long>(p.n_tiles) * blockIdx.x / p.ctas_per_head);
+  const int t1 =
+      static_cast<int>(static_cast<long long>(p.n_tiles) * (blockIdx.x + 1) / p.ctas_per_head);
+  const int n = t1 - t0;
+
+  if (warp == 0) {
+    tmem_alloc(&bar->tmem_base, 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 32) {
+    mbar_init(&bar->c_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->x_full[s], 1);
+      mbar_init(&bar->x_empty[s], 1);
+      mbar_init(&bar->s_full[s], 1);
+      mbar_init(&bar->s_empty[s], 128);
+    }
+    mbar_init(&bar->drain, 1);
+    bar->abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int c = tid; c < p.C; c += kAsgThreads)
+    sNorm[c] = p.norms[static_cast<size_t>(bh) * p.C + c];
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == kAsgProducer) {
+    if (lane_id() == 0 && n > 0) {
+      mbar_arrive_expect_tx(&bar->c_full, static_cast<uint32_t>(p.C * D * 2));
+      for (int pn = 0; pn < Cf::kPanels; ++pn)
+        tma_load_3d(sC + pn * Cf::kCPanel, &p.tm_c, &bar->c_full, pn * 64, 0, bh);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(&bar->x_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&bar->x_full[st], Cf::kXBytes);
+        for (int pn = 0; pn < Cf::kPanels; ++pn)
+          tma_load_3d(sX + st * Cf::kXBytes + pn * Cf::kXPanel, &p.tm_x, &bar->x_full[st],
+                      pn * 64, (t0 + j) * 128, bh);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        // let every copy started here land before the CTA retires
+        long long tw = clock64();
+        while (!mbar_try_wait(&bar->c_full, 0) && clock64() - tw < kWaitLimitCycles) {
+        }
+        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
+          tw = clock64();
+          while (!mbar_try_wait(&bar->x_full[j & 1], (j >> 1) & 1) &&
+                 clock64() - tw < kWaitLimitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == kAsgMma) {
+    if (lane_id() == 0 && n > 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, p.C, false, false);
+      const uint32_t x_addr = smem_u32(sX), c_addr = smem_u32(sC);
+      bool ok = mbar_wait(&bar->c_full, 0, abort_flag, p.status);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(&bar->x_full[st], (j >> 1) & 1, abort_flag, p.status)) break;
+        if (!mbar_wait(&bar->s_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t s_col = tmem + st * kMaxC;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          mma_bf16_ss(s_col, sdesc_sw128(x_addr + st * Cf::kXBytes + (kk >> 2) * Cf::kXPanel + off, 16, 1024),
+                      sdesc_sw128(c_addr + (kk >> 2) * Cf::kCPanel + off, 16, 1024), idesc,
+                      kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar->s_full[st]);
+        tc_commit(&bar->x_empty[st]);
+      }
+      if (*abort_flag) {
+        tc_commit(&bar->drain);
+        long long tw = clock64();
+        while (!mbar_try_wait(&bar->drain, 0) && clock64() - tw < kWaitLimitCycles) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ argmin
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int j = 0; j < n; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&bar->s_full[st], (j >> 1) & 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      float best = INFINITY;
+      int best_c = 0;
+      for (int ch = 0; ch < p.C / 32; ++ch) {
+        uint32_t s[32];
+        tmem_ld_32x32b_x32(lane_base + st * kMaxC + ch * 32, s);
+        tmem_ld_wait();
+        reg_fence(s);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float dist = fmaf(-2.0f, u2f(s[i]), sNorm[ch * 32 + i]);
+          if (dist < best) {  // strict: ties keep the smaller index
+            best = dist;
+            best_c = ch * 32 + i;
+          }
+        }
+      }
+      if (p.C % 32 != 0) {
+        // the last 16 columns of a C that is a multiple of 16 but not of 32
+        uint32_t s[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
+              "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]),
+              "=r"(s[12]), "=r"(s[13]), "=r"(s[14]), "=r"(s[15])
+            : "r"(lane_base + st * kMaxC + (p.C / 32) * 32)
+            : "memory");
+        tmem_ld_wait();
+        reg_fence(s);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = (p.C / 32) * 32 + i;
+          const float dist = fmaf(-2.0f, u2f(s[i]), sNorm[c]);
+          if (dist < best) {
+            best = dist;
+            best_c = c;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->s_empty[st]);
+      const int row = (t0 + j) * 128 + tid;
+      if (row < p.N) p.assign[static_cast<size_t>(bh) * p.N + row] = best_c;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// centroids (fp32) -> bf16 copy and squared norms of the bf16 values (fp32,
+// channel order). One warp per centroid.
+__global__ void kmeans_prep_kernel(const float* __restrict__ cent, int32_t rows, int32_t D,
+                                   svg_bf16* __restrict__ cent_bf16, float* __restrict__ norms) {
+  const int r = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  float acc = 0.0f;
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    const float x = cent[static_cast<size_t>(r) * D + c0 + lane];
+    const uint32_t b = pack_bf16x2(x, 0.0f) & 0xffffu;  // round to nearest even
+    cent_bf16[static_cast<size_t>(r) * D + c0 + lane] = static_cast<svg_bf16>(b);
+    const float xb = __uint_as_float(b << 16);
+    // fixed order: lane partials, then the warp's lanes in order
+    acc = fmaf(xb, xb, acc);
+  }
+  float tot = 0.0f;
+  for (int l = 0; l < 32; ++l) tot += __shfl_sync(0xffffffffu, acc, l);
+  if (lane == 0) norms[r] = tot;
+}
+
+// initial centroids: row floor(c * N / C) of each head
+__global__ void kmeans_init_kernel(const svg_bf16* __restrict__ x, int32_t N, int32_t D,
+                                   int32_t C, float* __restrict__ cent) {
+  const int bh = blockIdx.y, c = blockIdx.x;
+  const int64_t row = static_cast<int64_t>(c) * N / C;
+  for (int i = threadIdx.x; i < D; i += blockDim.x)
+    cent[(static_cast<size_t>(bh) * C + c) * D + i] =
+        __uint_as_float(static_cast<uint32_t>(x[(static_cast<size_t>(bh) * N + row) * D + i]) << 16);
+}
+
+// ------------------------------------------------------------ stable sort
+constexpr int kSortRows = 1024;  // rows per sort block
+
+// hist[bh][blk][c] = rows of block blk in cluster c
+__global__ void sort_hist_kernel(const int32_t* __restrict__ assign, int32_t N, int32_t C,
+                                 int32_t nblk, int32_t* __restrict__ hist, int* status) {
+  extern __shared__ int cnt[];
+  const int bh = blockIdx.y, blk = blockIdx.x;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) cnt[c] = 0;
+  __syncthreads();
+  const int r0 = blk * kSortRows, r1 = min(N, r0 + kSortRows);
+  for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+    const int a = assign[static_cast<size_t>(bh) * N + r];
+    if (a >= 0 && a < C) atomicAdd(&cnt[a], 1);
+    else atomicOr(status, kDevErrBounds);
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x)
+    hist[(static_cast<size_t>(bh) * nblk + blk) * C + c] = cnt[c];
+}
+
+// Per head: offsets[c] = rows in clusters < c; hist becomes each block's first
+// sorted position per cluster (offsets[c] + rows of earlier blocks in c).
+__global__ void sort_scan_kernel(int32_t* __restrict__ hist, int32_t N, int32_t C, int32_t nblk,
+                                 int32_t* __restrict__ offsets) {
+  extern __shared__ int tot[];
+  const int bh = blockIdx.x;
+  int32_t* h = hist + static_cast<size_t>(bh) * nblk * C;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    int run = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int v = h[static_cast<size_t>(b) * C + c];
+      h[static_cast<size_t>(b) * C + c] = run;
+      run += v;
+    }
+    tot[c] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int c = 0; c < C; ++c) {
+      const int v = tot[c];
+      tot[c] = run;
+      offsets[static_cast<size_t>(bh) * (C + 1) + c] = run;
+      run += v;
+    }
+    offsets[static_cast<size_t>(bh) * (C + 1) + C] = run;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x)
+    for (int b = 0; b < nblk; ++b) h[static_cast<size_t>(b) * C + c] += tot[c];
+}
+
+// One warp per block: walks its rows in order, 32 at a time, and gives each
+// the next free sorted position of its cluster (stable).
+__global__ void sort_rank_kernel(const int32_t* __restrict__ assign, const int32_t* __restrict__ hist,
+                                 int32_t N, int32_t C, int32_t nblk, int32_t* __restrict__ order) {
+  extern __shared__ int next[];
+  const int bh = blockIdx.y, blk = blockIdx.x;
+  const int lane = threadIdx.x;
+  for (int c = lane; c < C; c += 32) next[c] = hist[(static_cast<size_t>(bh) * nblk + blk) * C + c];
+  __syncwarp();
+  const int r0 = blk * kSortRows, r1 = min(N, r0 + kSortRows);
+  for (int base = r0; base < r1; base += 32) {
+    const int r = base + lane;
+    int a = r < r1 ? assign[static_cast<size_t>(bh) * N + r] : -1;
+    if (a >= C) a = -1;  // flagged by the histogram
+    const unsigned live = __ballot_sync(0xffffffffu, a >= 0);
+    const unsigned peers = __match_any_sync(0xffffffffu, a) & live;
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int pos = 0;
+    if (a >= 0) pos = next[a] + rank;
+    __syncwarp();
+    if (a >= 0 && rank == 0) next[a] += __popc(peers);
+    __syncwarp();
+    if (a >= 0) order[static_cast<size_t>(bh) * N + pos] = r;
+  }
+}
+
+// ------------------------------------------------------------ update
+// One warp per (bh, c): the mean of the members (sorted order) in fp32.
+template <int D>
+__global__ void kmeans_update_kernel(const svg_bf16* __restrict__ x, const int32_t* __restrict__ order,
+                                     const int32_t* __restrict__ offsets, int32_t N, int32_t C,
+                                     int32_t rows, const float* __restrict__ c_in,
+                                     float* __restrict__ c_out) {
+  constexpr int kPer = D / 32;  // channels per lane
+  const int gw = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows) return;
+  const int bh = gw / C, c = gw - bh * C;
+  const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
+  const int p0 = off[c], p1 = off[c + 1];
+  float acc[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+  for (int pos = p0; pos < p1; ++pos) {
+    const int r = order[static_cast<size_t>(bh) * N + pos];
+    const svg_bf16* src = x + (static_cast<size_t>(bh) * N + r) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(src);
+      acc[0] += __uint_as_float(u.x << 16);
+      acc[1] += __uint_as_float(u.x & 0xffff0000u);
+      acc[2] += __uint_as_float(u.y << 16);
+      acc[3] += __uint_as_float(u.y & 0xffff0000u);
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+      acc[0] += __uint_as_float(u << 16);
+      acc[1] += __uint_as_float(u & 0xffff0000u);
+    }
+  }
+  float* dst = c_out + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+  const float* prev = c_in + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+  const int cnt = p1 - p0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i)
+    dst[i] = cnt > 0 ? __fdiv_rn(acc[i], static_cast<float>(cnt)) : prev[i];
+}
+
+// ------------------------------------------------------------ selection
+// One CTA per (bh, query cluster a); thread b per key cluster.
+// With disp != nullptr (SVG-EAR), a skipped cluster is kept anyway when its
+// error estimate w_b * disp_b exceeds tau.
+__global__ void select_kernel(const float* __restrict__ cq, const float* __restrict__ ck,
+                              const int32_t* __restrict__ offsets_k, int32_t D, int32_t Cq,
+                              int32_t Ck, float scale, float top_p, const float* __restrict__ disp,
+                              float tau, uint32_t* __restrict__ sel) {
+  extern __shared__ float w[];  // [Ck] weights, then [32] reduction slots
+  float* red = w + Ck;
+  const int a = blockIdx.x, bh = blockIdx.y;
+  const int b = threadIdx.x;
+  const int lane = b & 31, wid = b >> 5, nw = blockDim.x >> 5;
+  const int words = (Ck + 31) / 32;
+  float z = -INFINITY;
+  int size = 0;
+  if (b < Ck) {
+    const int32_t* off = offsets_k + static_cast<size_t>(bh) * (Ck + 1);
+    size = off[b + 1] - off[b];
+    if (size > 0) {
+      const float* x = cq + (static_cast<size_t>(bh) * Cq + a) * D;
+      const float* y = ck + (static_cast<size_t>(bh) * Ck + b) * D;
+      float dot = 0.0f;
+      for (int i = 0; i < D; ++i) dot = fmaf(x[i], y[i], dot);
+      z = fmaf(scale, dot, logf(static_cast<float>(size)));
+    }
+  }
+  // block max
+  float m = z;
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[wid] = m;
+  __syncthreads();
+  m = -INFINITY;
+  for (int i = 0; i < nw; ++i) m = fmaxf(m, red[i]);
+  __syncthreads();
+  const float e = (b < Ck && size > 0) ? expf(z - m) : 0.0f;
+  // block sum in a fixed order
+  float s = e;
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red[wid] = s;
+  __syncthreads();
+  float tot = 0.0f;
+  for (int i = 0; i < nw; ++i) tot += red[i];
+  const float wb = e / tot;
+  if (b < Ck) w[b] = wb;
+  __syncthreads();
+  bool keep = false;
+  if (b < Ck && size > 0) {
+    // weight of the clusters ranked before b (descending weight, ties by index)
+    float before = 0.0f;
+    for (int i = 0; i < Ck; ++i) {
+      const float wi = w[i];
+      if (wi > wb || (wi == wb && i < b)) before += wi;
+    }
+    keep = before < top_p;
+    if (!keep && disp != nullptr) keep = wb * disp[static_cast<size_t>(bh) * Ck + b] > tau;
+  }
+  const unsigned bits = __ballot_sync(0xffffffffu, keep);
+  if (lane == 0 && wid < words) sel[(static_cast<size_t>(bh) * Cq + a) * words + wid] = bits;
+}
+
+// ------------------------------------------------------------ tile CSR
+constexpr int kTileWarps = 4;
+constexpr int kMaxSelWords = 32;    // Ck <= 1024
+constexpr int kMaxTileWords = 128;  // key tiles <= 4096
+
+// The key tiles of query tile r of head bh, as a bitmap in `tiles` (the
+// warp's shared words). Query clusters present in the tile: the clusters of
+// its first and last sorted positions and all between them.
+__device__ void tile_key_bitmap(const int32_t* __restrict__ offq, const int32_t* __restrict__ offk,
+                                const uint32_t* __restrict__ sel_bh, int32_t N, int32_t Cq,
+                                int32_t Ck, int32_t bq, int32_t bk, int32_t nkb, int r,
+                                uint32_t* keep, uint32_t* tiles) {
+  const int lane = threadIdx.x & 31;
+  const int sw = (Ck + 31) / 32, tw = (nkb + 31) / 32;
+  const int p0 = r * bq, p1 = min(N, p0 + bq) - 1;
+  // cluster of a sorted position: the last a with offq[a] <= pos
+  auto cluster_at = [&](int pos) {
+    int lo = 0, hi = Cq - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (offq[mid] <= pos) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  const int a0 = cluster_at(p0), a1 = cluster_at(p1);
+  for (int i = lane; i < sw; i += 32) {
+    uint32_t m = 0;
+    for (int a = a0; a <= a1; ++a)  // clusters with no position in the tile do not count
+      if (offq[a + 1] > offq[a]) m |= sel_bh[static_cast<size_t>(a) * sw + i];
+    keep[i] = m;
+  }
+  for (int i = lane; i < tw; i += 32) tiles[i] = 0;
+  __syncwarp();
+  for (int b = lane; b < Ck; b += 32) {
+    if (!((keep[b >> 5] >> (b & 31)) & 1u)) continue;
+    const int k0 = offk[b], k1 = offk[b + 1];
+    if (k1 <= k0) continue;
+    for (int t = k0 / bk; t <= (k1 - 1) / bk; ++t) atomicOr(&tiles[t >> 5], 1u << (t & 31));
+  }
+  __syncwarp();
+}
+
+__global__ void tile_count_kernel(const int32_t* __restrict__ offsets_q,
+                                  const int32_t* __restrict__ offsets_k,
+                                  const uint32_t* __restrict__ sel, int32_t BH, int32_t N,
+                                  int32_t Cq, int32_t Ck, int32_t bq, int32_t bk, int32_t nqb,
+                                  int32_t nkb, int32_t* __restrict__ counts) {
+  __shared__ uint32_t keep[kTileWarps][kMaxSelWords];
+  __shared__ uint32_t tiles[kTileWarps][kMaxTileWords];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kTileWarps + w;
+  if (row >= BH * nqb) return;
+  const int bh = row / nqb, r = row - bh * nqb;
+  const int sw = (Ck + 31) / 32, tw = (nkb + 31) / 32;
+  tile_key_bitmap(offsets_q + static_cast<size_t>(bh) * (Cq + 1),
+                  offsets_k + static_cast<size_t>(bh) * (Ck + 1),
+                  sel + static_cast<size_t>(bh) * Cq * sw, N, Cq, Ck, bq, bk, nkb, r, keep[w],
+                  tiles[w]);
+  int c = 0;
+  for (int i = lane; i < tw; i += 32) c += __popc(tiles[w][i]);
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) counts[row] = c;
+}
+
+// row_ptr[0] = 0, row_ptr[i+1] = row_ptr[i] + counts[i] (one CTA, fixed order)
+__global__ void tile_scan_kernel(const int32_t* __restrict__ counts, int32_t rows,
+                                 int32_t* __restrict__ row_ptr) {
+  __shared__ int32_t part[1024];
+  const int t = threadIdx.x, nt = blockDim.x;
+  const int per = (rows + nt - 1) / nt;
+  const int i0 = t * per, i1 = min(rows, i0 + per);
+  int32_t s = 0;
+  for (int i = i0; i < i1; ++i) s += counts[i];
+  part[t] = s;
+  __syncthreads();
+  if (t == 0) {
+    int32_t run = 0;
+    for (int i = 0; i < nt; ++i) {
+      const int32_t v = part[i];
+      part[i] = run;
+      run += v;
+    }
+    row_ptr[rows] = run;
+  }
+  __syncthreads();
+  int32_t run = part[t];
+  for (int i = i0; i < i1; ++i) {
+    row_ptr[i] = run;
+    run += counts[i];
+  }
+}
+
+__global__ void tile_fill_kernel(const int32_t* __restrict__ offsets_q,
+                                 const int32_t* __restrict__ offsets_k,
+                                 const uint32_t* __restrict__ sel, int32_t BH, int32_t N, int32_t Cq,
+                                 int32_t Ck, int32_t bq, int32_t bk, int32_t nqb, int32_t nkb,
+                                 const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+                                 int64_t capacity, int* status) {
+  __shared__ uint32_t keep[kTileWarps][kMaxSelWords];
+  __shared__ uint32_t tiles[kTileWarps][kMaxTileWords];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kTileWarps + w;
+  if (row >= BH * nqb) return;
+  const int bh = row / nqb, r = row - bh * nqb;
+  const int sw = (Ck + 31) / 32, tw = (nkb + 31) / 32;
+  tile_key_bitmap(offsets_q + static_cast<size_t>(bh) * (Cq + 1),
+                  offsets_k + static_cast<size_t>(bh) * (Ck + 1),
+                  sel + static_cast<size_t>(bh) * Cq * sw, N, Cq, Ck, bq, bk, nkb, r, keep[w],
+                  tiles[w]);
+  int64_t pos = row_ptr[row];
+  for (int i0 = 0; i0 < tw; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t bits = i < tw ? tiles[w][i] : 0u;
+    const int c = __popc(bits);
+    int incl = c;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int64_t p = pos + incl - c;
+    for (uint32_t m = bits; m; m &= m - 1) {
+      const int t = 32 * i + __ffs(m) - 1;
+      if (p < capacity) col_idx[p] = t;
+      else atomicOr(status, kDevErrBounds);
+      ++p;
+    }
+    pos += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+// ------------------------------------------------------------ row permutation
+// gather: y[bh, pos] = x[bh, order[bh, pos]];  scatter: y[bh, order[bh, pos]] = x[bh, pos]
+template <bool kScatter>
+__global__ void permute_rows_kernel(const svg_bf16* __restrict__ x, const int32_t* __restrict__ order,
+                                    int32_t BH, int32_t N, int32_t D, svg_bf16* __restrict__ y,
+                                    int* status) {
+  const int vec = D / 8;  // 16-byte vectors per row
+  const int64_t total = static_cast<int64_t>(BH) * N * vec;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t rowi = i / vec;
+    const int v = static_cast<int>(i - rowi * vec);
+    const int64_t bh = rowi / N;
+    const int pos = static_cast<int>(rowi - bh * N);
+    const int r = order[rowi];
+    if (r < 0 || r >= N) {
+      atomicOr(status, kDevErrBounds);
+      continue;
+    }
+    const int64_t src = kScatter ? rowi : bh * N + r;
+    const int64_t dst = kScatter ? bh * N + r : rowi;
+    reinterpret_cast<uint4*>(y + dst * D)[v] = reinterpret_cast<const uint4*>(x + src * D)[v];
+    (void)pos;
+  }
+}
+
+// ------------------------------------------------------------ SVG-EAR
+// Per key cluster (one warp per (bh, b)), over its members in sorted order:
+// vbar = the fp32 mean value, disp = sqrt(mean over members and channels of
+// (v - vbar)^2); an empty cluster gets zeros.
+template <int D>
+__global__ void cluster_stats_kernel(const svg_bf16* __restrict__ v, const int32_t* __restrict__ order,
+                                     const int32_t* __restrict__ offsets, int32_t N, int32_t C,
+                                     int32_t rows, float* __restrict__ vbar,
+                                     float* __restrict__ disp) {
+  constexpr int kPer = D / 32;
+  const int gw = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows) return;
+  const int bh = gw / C, c = gw - bh * C;
+  const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
+  const int p0 = off[c], p1 = off[c + 1];
+  auto load = [&](int pos, float (&x)[kPer]) {
+    const int r = order[static_cast<size_t>(bh) * N + pos];
+    const svg_bf16* src = v + (static_cast<size_t>(bh) * N + r) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(src);
+      x[0] = __uint_as_float(u.x << 16);
+      x[1] = __uint_as_float(u.x & 0xffff0000u);
+      x[2] = __uint_as_float(u.y << 16);
+      x[3] = __uint_as_float(u.y & 0xffff0000u);
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+      x[0] = __uint_as_float(u << 16);
+      x[1] = __uint_as_float(u & 0xffff0000u);
+    }
+  };
+  float mean[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) mean[i] = 0.0f;
+  for (int pos = p0; pos < p1; ++pos) {
+    float x[kPer];
+    load(pos, x);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) mean[i] += x[i];
+  }
+  const int cnt = p1 - p0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) mean[i] = cnt > 0 ? __fdiv_rn(mean[i], static_cast<float>(cnt)) : 0.0f;
+  float sq = 0.0f;
+  for (int pos = p0; pos < p1; ++pos) {
+    float x[kPer];
+    load(pos, x);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) sq = fmaf(x[i] - mean[i], x[i] - mean[i], sq);
+  }
+  float tot = 0.0f;
+  for (int l = 0; l < 32; ++l) tot += __shfl_sync(0xffffffffu, sq, l);
+  float* dst = vbar + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) dst[i] = mean[i];
+  if (lane == 0)
+    disp[static_cast<size_t>(bh) * C + c] =
+        cnt > 0 ? sqrtf(__fdiv_rn(tot, static_cast<float>(cnt) * D)) : 0.0f;
+}
+
+// fp32 [rows, D] -> bf16 [rows, D] (round to nearest even)
+__global__ void to_bf16_kernel(const float* __restrict__ x, int64_t n, svg_bf16* __restrict__ y) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    y[i] = static_cast<svg_bf16>(pack_bf16x2(x[i], 0.0f) & 0xffffu);
+}
+
+// Centroid compensation of one sorted query tile (128 rows) of head bh:
+//   bias_b = log2(n_b), n_b = keys of cluster b outside the tile's computed key
+//            tiles (-inf when none);
+//   S = Q kbar^T (tcgen05, 128 x Ck), z_b = S_b * scale * log2(e) + bias_b,
+//   P = 2^(z - max z) (bf16, in tensor memory), O_c = P vbar (tcgen05);
+// then merged with the block-sparse output of the same rows through its
+// log-sum-exp: O = (O_s e^lse + O_c 2^m) / (e^lse + sum P 2^m), in place.
+constexpr int kEarThreads = 192;  // warps 0-3 softmax / merge, 4 producer, 5 MMA
+constexpr int kEarMaxTiles = 4096;
+
+struct EarBarriers {
+  uint64_t c_full, q_full, s_full, p_full, o_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  uint32_t tiles[kEarMaxTiles / 32];
+};
+
+template <int D>
+struct EarCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kCPanel = kMaxC * 128;  // up to 256 centroid rows x 128 B
+  static constexpr int kCBytes = kPanels * kCPanel;
+  static constexpr int kQPanel = 128 * 128;
+  static constexpr int kQBytes = kPanels * kQPanel;
+  static constexpr int kOffK = 0;               // kbar (K-major operand of S)
+  static constexpr int kOffV = kOffK + kCBytes;  // vbar (MN-major operand of O)
+  static constexpr int kOffQ = kOffV + kCBytes;
+  static constexpr int kOffBias = kOffQ + kQBytes;
+  static constexpr int kOffBar = kOffBias + kMaxC * 4;
+  static constexpr int kBarBytes = (static_cast<int>(sizeof(EarBarriers)) + 127) / 128 * 128;
+  static constexpr int kUsed = kOffBar + kBarBytes + 1024;
+  static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
+  static constexpr uint32_t kColS = 0, kColO = 256;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+};
+
+struct __align__(64) EarParams {
+  CUtensorMap tm_q;   // sorted queries [BH, N, D], box (64, 128)
+  CUtensorMap tm_kb;  // kbar bf16 [BH, C, D], box (64, C)
+  CUtensorMap tm_vb;  // vbar bf16 [BH, C, D], box (64, C)
+  const int32_t* offsets_k;  // [BH, C+1]
+  const int32_t* row_ptr;    // [BH*nqb+1]
+  const int32_t* col_idx;
+  svg_bf16* os;              // [BH, N, D] sorted sparse output, overwritten
+  const float* lse;          // [BH, N] natural log
+  int* status;
+  int32_t N, C, bk, nqb, nkb;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __grid_constant__ EarParams p) {
+  using Cf = EarCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem + Cf::kOffK;
+  uint8_t* sV = smem + Cf::kOffV;
+  uint8_t* sQ = smem + Cf::kOffQ;
+  float* sBias = reinterpret_cast<float*>(smem + Cf::kOffBias);
+  EarBarriers* bar = reinterpret_cast<EarBarriers*>(smem + Cf::kOffBar);
+  volatile int* abort_flag = &bar->abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int r = blockIdx.x, bh = blockIdx.y;
+
+  if (warp == 0) {
+    tmem_alloc(&bar->tmem_base, 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 32) {
+    mbar_init(&bar->c_full, 1);
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->p_full, 128);
+    mbar_init(&bar->o_full, 1);
+    mbar_init(&bar->drain, 1);
+    bar->abort_flag = 0;
+    fence_mbar_init();
+  }
+  // the tile's computed key tiles as a bitmap
+  const int tw = (p.nkb + 31) / 32;
+  for (int i = tid; i < tw; i += kEarThreads) bar->tiles[i] = 0u;
+  __syncthreads();
+  const int row = bh * p.nqb + r;
+  const int c0 = p.row_ptr[row], c1 = p.row_ptr[row + 1];
+  for (int i = c0 + tid; i < c1; i += kEarThreads) {
+    const int t = p.col_idx[i];
+    if (t >= 0 && t < p.nkb) atomicOr(&bar->tiles[t >> 5], 1u << (t & 31));
+    else atomicOr(p.status, kDevErrBounds);
+  }
+  __syncthreads();
+  // bias_b = log2 of the cluster's uncovered keys
+  const int32_t* off = p.offsets_k + static_cast<size_t>(bh) * (p.C + 1);
+  for (int b = tid; b < p.C; b += kEarThreads) {
+    const int k0 = off[b], k1 = off[b + 1];
+    int covered = 0;
+    if (k1 > k0) {
+      for (int t = k0 / p.bk; t <= (k1 - 1) / p.bk; ++t) {
+        if ((bar->tiles[t >> 5] >> (t & 31)) & 1u) {
+          const int lo = max(k0, t * p.bk), hi = min(k1, (t + 1) * p.bk);
+          covered += hi - lo;
+        }
+      }
+    }
+    const int n = k1 - k0 - covered;
+    sBias[b] = n > 0 ? __log2f(static_cast<float>(n)) : -INFINITY;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 4) {
+    if (lane_id() == 0) {
+      mbar_arrive_expect_tx(&bar->c_full, static_cast<uint32_t>(2 * p.C * D * 2));
+      for (int pn = 0; pn < Cf::kPanels; ++pn) {
+        tma_load_3d(sK + pn * Cf::kCPanel, &p.tm_kb, &bar->c_full, pn * 64, 0, bh);
+        tma_load_3d(sV + pn * Cf::kCPanel, &p.tm_vb, &bar->c_full, pn * 64, 0, bh);
+      }
+      mbar_arrive_expect_tx(&bar->q_full, Cf::kQBytes);
+      for (int pn = 0; pn < Cf::kPanels; ++pn)
+        tma_load_3d(sQ + pn * Cf::kQPanel, &p.tm_q, &bar->q_full, pn * 64, r * 128, bh);
+      long long tw0 = clock64();
+      // wait for our own copies before the CTA may retire (bounded)
+      while (!(mbar_try_wait(&bar->c_full, 0) && mbar_try_wait(&bar->q_full, 0)) &&
+             clock64() - tw0 < kWaitLimitCycles) {
+      }
+    }
+  } else if (warp == 5) {
+    if (lane_id() == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, p.C, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      bool ok = mbar_wait(&bar->c_full, 0, abort_flag, p.status) &&
+                mbar_wait(&bar->q_full, 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk & 3) * 32;
+          mma_bf16_ss(tmem + Cf::kColS, sdesc_sw128(q_addr + (kk >> 2) * Cf::kQPanel + o, 16, 1024),
+                      sdesc_sw128(k_addr + (kk >> 2) * Cf::kCPanel + o, 16, 1024), idesc_s,
+                      kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar->s_full);
+        ok = mbar_wait(&bar->p_full, 0, abort_flag, p.status);
+      }
+      if (ok) {
+        tc_fence_after();
+        for (int kk = 0; kk < p.C / 16; ++kk)
+          mma_bf16_ts(tmem + Cf::kColO, tmem + Cf::kColS + kk * 8,
+                      sdesc_sw128(v_addr + kk * 16 * 128, Cf::kCPanel, 1024), idesc_o,
+                      kk > 0 ? 1u : 0u);
+        tc_commit(&bar->o_full);
+      }
+      if (*abort_flag) {
+        tc_commit(&bar->drain);
+        long long tw0 = clock64();
+        while (!mbar_try_wait(&bar->drain, 0) && clock64() - tw0 < kWaitLimitCycles) {
+        }
+      }
+    }
+  } else {
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    bool ok = mbar_wait(&bar->s_full, 0, abort_flag, p.status);
+    float m = -INFINITY, den = 0.0f;
+    if (ok) {
+      tc_fence_after();
+      for (int ch = 0; ch < p.C / 32; ++ch) {
+        uint32_t s[32];
+        tmem_ld_32x32b_x32(lane_base + Cf::kColS + ch * 32, s);
+        tmem_ld_wait();
+        reg_fence(s);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          m = fmaxf(m, fmaf(u2f(s[i]), p.scale_log2, sBias[ch * 32 + i]));
+      }
+      if (p.C % 32 != 0) {
+        uint32_t s[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
+              "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]),
+              "=r"(s[12]), "=r"(s[13]), "=r"(s[14]), "=r"(s[15])
+            : "r"(lane_base + Cf::kColS + (p.C / 32) * 32)
+            : "memory");
+        tmem_ld_wait();
+        reg_fence(s);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          m = fmaxf(m, fmaf(u2f(s[i]), p.scale_log2, sBias[(p.C / 32) * 32 + i]));
+      }
+      const float mu = m == -INFINITY ? 0.0f : m;
+      // P in 16-column chunks: S columns [16 ch, 16 ch + 16) -> P columns [8 ch, 8 ch + 8)
+      for (int ch = 0; ch < p.C / 16; ++ch) {
+        uint32_t s[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
+              "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]),
+              "=r"(s[12]), "=r"(s[13]), "=r"(s[14]), "=r"(s[15])
+            : "r"(lane_base + Cf::kColS + ch * 16)
+            : "memory");
+        tmem_ld_wait();
+        reg_fence(s);
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int b = ch * 16 + 2 * i;
+          const float p0 = fast_exp2(fmaf(u2f(s[2 * i]), p.scale_log2, sBias[b]) - mu);
+          const float p1 = fast_exp2(fmaf(u2f(s[2 * i + 1]), p.scale_log2, sBias[b + 1]) - mu);
+          den += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        // P of these 16 clusters overwrites S columns the loop has already read
+        tmem_st_32x32b_x8(lane_base + Cf::kColS + ch * 8, pk);
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    mbar_arrive(&bar->p_full);
+    if (ok) ok = mbar_wait(&bar->o_full, 0, abort_flag, p.status);
+    tc_fence_after();
+    // merge with the sparse output of this row
+    const int qrow = r * 128 + tid;
+    if (__all_sync(0xffffffffu, ok) && qrow < p.N) {
+      const size_t ro = static_cast<size_t>(bh) * p.N + qrow;
+      const float lse2 = p.lse[ro] * 1.4426950408889634f;
+      const float M = fmaxf(lse2, m);
+      const float a = lse2 == -INFINITY ? 0.0f : fast_exp2(lse2 - M);
+      const float c = m == -INFINITY ? 0.0f : fast_exp2(m - M);
+      const float tot = a + den * c;
+      const float inv = tot > 0.0f ? 1.0f / tot : 0.0f;  // no key at all: O = 0
+      svg_bf16* orow = p.os + ro * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(lane_base + Cf::kColO + ch * 32, o);
+        tmem_ld_wait();
+        reg_fence(o);
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        uint32_t pk[16];
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const uint4 in = dst[v4];
+          const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e = 8 * v4 + 2 * i;
+            const float s0 = __uint_as_float(w[i] << 16), s1 = __uint_as_float(w[i] & 0xffff0000u);
+            pk[4 * v4 + i] = pack_bf16x2((s0 * a + u2f(o[e]) * c) * inv,
+                                         (s1 * a + u2f(o[e + 1]) * c) * inv);
+          }
+        }
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+    } else if (!ok && tid == 0) {
+      atomicOr(p.status, kDevErrTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+size_t kmeans_workspace_bytes(int32_t BH, int32_t N, int32_t D, int32_t C) {
+  const size_t nblk = (static_cast<size_t>(N) + kSortRows - 1) / kSortRows;
+  size_t b = 0;
+  auto add = [&](size_t n) { b = (b + 255) / 256 * 256 + n; };
+  add(static_cast<size_t>(BH) * C * D * 2);        // bf16 centroids
+  add(static_cast<size_t>(BH) * C * 4);            // norms
+  add(static_cast<size_t>(BH) * nblk * C * 4);     // sort histograms
+  add(static_cast<size_t>(BH) * C * D * 4);        // the other centroid buffer
+  return (b + 255) / 256 * 256;
+}
+
+namespace {
+struct KWs {
+  svg_bf16* cb;
+  float* norms;
+  int32_t* hist;
+  float* cent2;
+};
+KWs carve(void* ws, int32_t BH, int32_t N, int32_t D, int32_t C) {
+  const size_t nblk = (static_cast<size_t>(N) + kSortRows - 1) / kSortRows;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t b = 0;
+  auto take = [&](size_t n) {
+    b = (b + 255) / 256 * 256;
+    uint8_t* p = base + b;
+    b += n;
+    return p;
+  };
+  KWs w;
+  w.cb = reinterpret_cast<svg_bf16*>(take(static_cast<size_t>(BH) * C * D * 2));
+  w.norms = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * C * 4));
+  w.hist = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nblk * C * 4));
+  w.cent2 = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * C * D * 4));
+  return w;
+}
+
+template <int D>
+cudaError_t launch_assign(int32_t BH, int32_t N, int32_t C, const svg_bf16* x, const KWs& w,
+                          int32_t* assign, int* status, cudaStream_t stream) {
+  using Cf = AsgCfg<D>;
+  AsgParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_tmap_bf16(&p.tm_x, x, D, N, BH, 128) || !make_tmap_bf16(&p.tm_c, w.cb, D, C, BH, C))
+    return cudaErrorInvalidValue;
+  p.norms = w.norms;
+  p.assign = assign;
+  p.status = status;
+  p.N = N;
+  p.C = C;
+  p.n_tiles = (N + 127) / 128;
+  // one wave of CTAs over all heads (148 SMs), at least one per head
+  int per = 148 / BH;
+  if (per > p.n_tiles) per = p.n_tiles;
+  if (per < 1) per = 1;
+  p.ctas_per_head = per;
+  auto kern = kmeans_assign_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(per, BH), kAsgThreads, Cf::kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_kmeans_assign(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
+                                 const float* centroids, int32_t* assign, void* ws, int* status,
+                                 cudaStream_t stream) {
+  const KWs w = carve(ws, BH, N, D, C);
+  const int rows = BH * C;
+  kmeans_prep_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(centroids, rows, D, w.cb, w.norms);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return D == 128 ? launch_assign<128>(BH, N, C, x, w, assign, status, stream)
+                  : launch_assign<64>(BH, N, C, x, w, assign, status, stream);
+}
+
+cudaError_t launch_cluster_sort(int32_t BH, int32_t N, int32_t C, const int32_t* assign,
+                                int32_t* order, int32_t* offsets, void* ws, int32_t D, int* status,
+                                cudaStream_t stream) {
+  const KWs w = carve(ws, BH, N, D, C);
+  const int nblk = (N + kSortRows - 1) / kSortRows;
+  const size_t sm = static_cast<size_t>(C) * sizeof(int);
+  sort_hist_kernel<<<dim3(nblk, BH), 256, sm, stream>>>(assign, N, C, nblk, w.hist, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sort_scan_kernel<<<BH, 256, sm, stream>>>(w.hist, N, C, nblk, offsets);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sort_rank_kernel<<<dim3(nblk, BH), 32, sm, stream>>>(assign, w.hist, N, C, nblk, order);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
+                                 const int32_t* order, const int32_t* offsets, const float* c_in,
+                                 float* c_out, cudaStream_t stream) {
+  const int rows = BH * C;
+  if (D == 128)
+    kmeans_update_kernel<128><<<(rows + 7) / 8, 256, 0, stream>>>(x, order, offsets, N, C, rows,
+                                                                 c_in, c_out);
+  else
+    kmeans_update_kernel<64><<<(rows + 7) / 8, 256, 0, stream>>>(x, order, offsets, N, C, rows,
+                                                                c_in, c_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kmeans(int32_t BH, int32_t N, int32_t D, int32_t C, int32_t iters,
+                          const svg_bf16* x, float* centroids, int32_t* assign, int32_t* order,
+                          int32_t* offsets, void* ws, int* status, cudaStream_t stream) {
+  const KWs w = carve(ws, BH, N, D, C);
+  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, centroids);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the iterations alternate between the caller's buffer and the workspace
+  // copy so that the last update lands in the caller's buffer
+  float* bufs[2] = {centroids, w.cent2};
+  int cur = 0;
+  if (iters % 2 == 1) {
+    e = cudaMemcpyAsync(w.cent2, centroids, static_cast<size_t>(BH) * C * D * 4,
+                        cudaMemcpyDeviceToDevice, stream);
+    if (e != cudaSuccess) return e;
+    cur = 1;
+  }
+  for (int it = 0; it < iters; ++it) {
+    if ((e = launch_kmeans_assign(BH, N, D, C, x, bufs[cur], assign, ws, status, stream)) !=
+        cudaSuccess)
+      return e;
+    if ((e = launch_cluster_sort(BH, N, C, assign, order, offsets, ws, D, status, stream)) !=
+        cudaSuccess)
+      return e;
+    if ((e = launch_kmeans_update(BH, N, D, C, x, order, offsets, bufs[cur], bufs[cur ^ 1],
+                                  stream)) != cudaSuccess)
+      return e;
+    cur ^= 1;
+  }
+  if (iters == 0) {
+    if ((e = launch_kmeans_assign(BH, N, D, C, x, centroids, assign, ws, status, stream)) !=
+        cudaSuccess)
+      return e;
+    return launch_cluster_sort(BH, N, C, assign, order, offsets, ws, D, status, stream);
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_select_clusters(int32_t BH, int32_t D, int32_t Cq, int32_t Ck, float scale,
+                                   float top_p, const float* cq, const float* ck,
+                                   const int32_t* offsets_k, const float* disp, float tau,
+                                   uint32_t* sel, cudaStream_t stream) {
+  const int threads = (Ck + 31) / 32 * 32;
+  const size_t sm = (static_cast<size_t>(Ck) + 32) * sizeof(float);
+  select_kernel<<<dim3(Cq, BH), threads, sm, stream>>>(cq, ck, offsets_k, D, Cq, Ck, scale, top_p,
+                                                      disp, tau, sel);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_csr(int32_t BH, int32_t N, int32_t Cq, int32_t Ck, int32_t bq, int32_t bk,
+                            const int32_t* offsets_q, const int32_t* offsets_k, const uint32_t* sel,
+                            int32_t* row_ptr, int32_t* col_idx, int64_t capacity, int32_t* counts,
+                            int* status, cudaStream_t stream) {
+  const int nqb = (N + bq - 1) / bq, nkb = (N + bk - 1) / bk;
+  const int rows = BH * nqb;
+  const int blocks = (rows + kTileWarps - 1) / kTileWarps;
+  tile_count_kernel<<<blocks, 32 * kTileWarps, 0, stream>>>(offsets_q, offsets_k, sel, BH, N, Cq,
+                                                            Ck, bq, bk, nqb, nkb, counts);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tile_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tile_fill_kernel<<<blocks, 32 * kTileWarps, 0, stream>>>(offsets_q, offsets_k, sel, BH, N, Cq, Ck,
+                                                           bq, bk, nqb, nkb, row_ptr, col_idx,
+                                                           capacity, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_rows(int32_t BH, int32_t N, int32_t D, const svg_bf16* x,
+                                const int32_t* order, svg_bf16* y, bool scatter, int* status,
+                                cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(BH) * N * (D / 8);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 16 * 148) blocks = 16 * 148;
+  if (scatter)
+    permute_rows_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, order, BH, N, D,
+                                                                                 y, status);
+  else
+    permute_rows_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, order, BH, N,
+                                                                                  D, y, status);
+  return cudaGetLastError();
+}
+
+}  // namespace svg
+
+namespace svg {
+
+cudaError_t launch_cluster_stats(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* v,
+                                 const int32_t* order, const int32_t* offsets, float* vbar,
+                                 float* disp, cudaStream_t stream) {
+  const int rows = BH * C;
+  if (D == 128)
+    cluster_stats_kernel<128><<<(rows + 7) / 8, 256, 0, stream>>>(v, order, offsets, N, C, rows,
+                                                                 vbar, disp);
+  else
+    cluster_stats_kernel<64><<<(rows + 7) / 8, 256, 0, stream>>>(v, order, offsets, N, C, rows,
+                                                                vbar, disp);
+  return cudaGetLastError();
+}
+
+size_t ear_workspace_bytes(int32_t BH, int32_t D, int32_t C) {
+  return (static_cast<size_t>(BH) * C * D * 2 * 2 + 255) / 256 * 256;
+}
+
+cudaError_t launch_ear_compensate(int32_t BH, int32_t N, int32_t D, int32_t C, int32_t bk,
+                                  float scale, const svg_bf16* qs, const float* kbar,
+                                  const float* vbar, const int32_t* offsets_k,
+                                  const int32_t* row_ptr, const int32_t* col_idx, svg_bf16* os,
+                                  const float* lse, void* ws, int* status, cudaStream_t stream) {
+  svg_bf16* kb = static_cast<svg_bf16*>(ws);
+  svg_bf16* vb = kb + static_cast<size_t>(BH) * C * D;
+  const int64_t n = static_cast<int64_t>(BH) * C * D;
+  to_bf16_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0,
+                   stream>>>(kbar, n, kb);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  to_bf16_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0,
+                   stream>>>(vbar, n, vb);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  EarParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_tmap_bf16(&p.tm_q, qs, D, N, BH, 128) || !make_tmap_bf16(&p.tm_kb, kb, D, C, BH, C) ||
+      !make_tmap_bf16(&p.tm_vb, vb, D, C, BH, C))
+    return cudaErrorInvalidValue;
+  p.offsets_k = offsets_k;
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.os = os;
+  p.lse = lse;
+  p.status = status;
+  p.N = N;
+  p.C = C;
+  p.bk = bk;
+  p.nqb = (N + 127) / 128;
+  p.nkb = (N + bk - 1) / bk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (D == 128) {
+    auto kern = ear_compensate_kernel<128>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  EarCfg<128>::kSmem)) != cudaSuccess)
+      return e;
+    kern<<<dim3(p.nqb, BH), kEarThreads, EarCfg<128>::kSmem, stream>>>(p);
+  } else {
+    auto kern = ear_compensate_kernel<64>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  EarCfg<64>::kSmem)) != cudaSuccess)
+      return e;
+    kern<<<dim3(p.nqb, BH), kEarThreads, EarCfg<64>::kSmem, stream>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace svg
