@@ -36,6 +36,9 @@ import svg_inputs as SI  # noqa: E402
 METRIC = "sparse-attn layer ms & TFLOPS (computed blocks) vs BF16 peak; speedup vs dense"
 UNIT = "TFLOP/s (computed blocks)"
 DEFAULT_WORKLOAD = SI.HUNYUAN.name
+# the semantic-aware (SVG2) measurement: clusters of queries and keys, Lloyd
+# iterations and the kept share of the centroid attention
+SVG2_CQ, SVG2_CK, SVG2_ITERS, SVG2_TOP_P = 256, 256, 10, 0.9
 
 
 def _peaks():
@@ -50,23 +53,39 @@ def _peaks():
             "source": "fallback"}
 
 
-def _captured_traffic():
-    """DRAM bytes per full-size attention launch from the committed ncu summary,
-    or None when the kernel sources changed since that capture."""
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def _sources_digest(files) -> str:
     import hashlib
-    path = os.path.join(ROOT, "profiles", "sparse_attention_pair_hunyuan_H4_d128.md")
-    srcs = [os.path.join(ROOT, "video_dit_spatial_b200", "csrc", f)
-            for f in ("attention.cu", "sm100.cuh")]
+    paths = [os.path.join(ROOT, "video_dit_spatial_b200", "csrc", f) for f in files]
+    return hashlib.sha256(b"".join(open(f, "rb").read() for f in paths)).hexdigest()[:16]
+
+
+def _captured_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per full-size launch of `kernel` on `workload`
+    from profiles/traffic.json (written from an ncu capture), or None when there
+    is no entry or the kernel's sources changed since that capture."""
     try:
-        text = open(path).read()
-        digest = hashlib.sha256(b"".join(open(f, "rb").read() for f in srcs)).hexdigest()[:16]
+        entries = json.load(open(TRAFFIC_JSON))
+    except (OSError, ValueError):
+        return None
+    e = entries.get(kernel)
+    if not e or e.get("workload") != workload:
+        return None
+    try:
+        if _sources_digest(e["sources"]) != e["sources_sha256_16"]:
+            return None
     except OSError:
         return None
-    fields = dict(line.strip().split(": ", 1) for line in text.splitlines()
-                  if line.strip().startswith(("traffic_bytes", "kernel_sources")))
-    if fields.get("kernel_sources_sha256_16") != digest:
-        return None
-    return int(fields["traffic_bytes_per_launch_full_size"])
+    return int(e["traffic_bytes_per_launch_full_size"])
+
+
+def percentiles(ms_list):
+    """p10 / p50 / p90 (linear interpolation) and the mean of a list of ms."""
+    a = np.asarray(ms_list, dtype=np.float64)
+    return {"p10": float(np.percentile(a, 10)), "p50": float(np.percentile(a, 50)),
+            "p90": float(np.percentile(a, 90)), "mean": float(a.mean()), "n": int(a.size)}
 
 
 def _dist_env():
@@ -195,6 +214,47 @@ def oracle_sample(wl, n_rows: int, heads, seed: int = 5):
     return elapsed, flops
 
 
+def oracle_components(wl, n_rows: int = 128, n_qblocks: int = 3):
+    """Times the oracle's other steps on bounded samples of the workload, with
+    a labelled extrapolation of each to the whole layer:
+      profiling  the full and both masked attentions, MSEs and label of one head
+                 on n_rows of its sampled rows (layer: n_samples rows x B*H heads);
+      masks      brute-force block-mask rows (OR over token pairs) of n_qblocks
+                 query blocks per pattern (layer: every query block, 2 patterns);
+      permute    the layout transformation of one head's Q (layer: Q, K, V and
+                 the inverse of O for every temporal head)."""
+    import oracle as O
+    kinds = SI.planted_head_kinds(wl)
+    h = kinds.index(1) if 1 in kinds else 0
+    q, k, v = (O.from_bf16_bits(t.view(torch.int16).numpy()) for t in SI.make_head(wl, 0, h))
+    rows = SI.sample_rows(wl).numpy()
+    sub = rows[np.linspace(0, rows.size - 1, min(n_rows, rows.size)).astype(np.int64)]
+    t0 = time.perf_counter()
+    O.profile_head(q, k, v, sub, wl.T, wl.P, wl.n_text, wl.spatial_band, wl.temporal_width,
+                   wl.scale)
+    t_prof = time.perf_counter() - t0
+    nqb = -(-wl.N // wl.block_q)
+    qbs = np.linspace(0, nqb - 1, n_qblocks).astype(np.int64)
+    t0 = time.perf_counter()
+    for kind in (O.MASK_SPATIAL, O.MASK_TEMPORAL):
+        O.block_mask_rows(kind, qbs, wl.T, wl.P, wl.n_text, wl.spatial_band, wl.temporal_width,
+                          wl.block_q, wl.block_k)
+    t_mask = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.permute(q, wl.T, wl.P, wl.n_text)
+    t_perm = time.perf_counter() - t0
+    n_temporal = wl.B * sum(kinds)
+    return {
+        "profiling": {"seconds": t_prof, "sample": f"1 head x {sub.size} sampled rows",
+                      "extrapolated_layer_s": t_prof * wl.n_samples / sub.size * wl.B * wl.H},
+        "block_masks": {"seconds": t_mask,
+                        "sample": f"{len(qbs)} query blocks x 2 patterns, brute force",
+                        "extrapolated_layer_s": t_mask * nqb / len(qbs)},
+        "permute": {"seconds": t_perm, "sample": "Q of 1 head",
+                    "extrapolated_layer_s": t_perm * 4 * n_temporal},
+    }
+
+
 def cpu_threads() -> int:
     try:
         import threadpoolctl
@@ -274,6 +334,13 @@ def run_capture(args, wl):
         "profile": lambda: fu.profile(q, k, v, rows),
         "permute": lambda: svg.svg_permute_qkv(g, q, k, v, ex.qp, ex.kp, ex.vp, ex.labels),
     }
+    if args.capture == "attention_fp8":
+        v8 = torch.empty(q.shape, dtype=torch.uint8, device="cuda")
+        v_scale = torch.empty(wl.B * wl.H * wl.d, dtype=torch.float32, device="cuda")
+        svg.svg_quantize_v_e4m3(g, v, ex.vp, ex.labels, v8, v_scale)
+        fns["attention_fp8"] = lambda: svg.svg_sparse_attention_fp8pv(
+            g, q, k, ex.qp, ex.kp, v8, v_scale, ex.labels, ex.masks[0].row_ptr,
+            ex.masks[0].col_idx, ex.masks[1].row_ptr, ex.masks[1].col_idx, o, ex.op)
     fn = fns[args.capture]
     for it in range(3):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -300,8 +367,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true")
+    ap.add_argument("--no-svg2", action="store_true")
     ap.add_argument("--capture", choices=["attention", "attention_fused", "attention_gathered",
-                                          "profile", "permute"],
+                                          "attention_fp8", "profile", "permute"],
                     help="small case for an ncu capture: run one kernel 3 times on the "
                          "workload with --heads heads, print per-launch ms, no JSON line")
     ap.add_argument("--heads", type=int, default=4)
@@ -358,16 +427,19 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
+    # one event before the first step and one after every step: the region's
+    # time (the barrier-bracketed total) and each step's own time
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
         step()
-    ev1.record(stream)
+        evs[i + 1].record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
-    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+    ms = max_over_ranks(evs[0].elapsed_time(evs[-1]) / args.steps, dist, dev)
+    step_pct = percentiles([evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)])
     # profile, finalize, 2 masks, attention, plus the layout passes: permute_qkv and
     # unpermute (explicit), permute of K and V (fused), none (gathered); plus the
     # profiling combine kernel when the key ranges are split (a workspace larger
@@ -376,20 +448,21 @@ def main():
     split = svg.svg_profile_workspace_bytes(g, wl.n_samples) > wl.B * wl.H * 2 * tiles * 4
     gpu_launches = ({"explicit": 7, "fused": 6, "gathered": 5}[layout] + int(split)) * args.steps
 
-    # per-kernel timing (events on the launch stream), then the dense baseline
+    # per-kernel timing: an event pair around every launch on the launch stream,
+    # after one untimed launch; p10 / p50 / p90 over the launches
     def time_fn(fn, reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         fn()
         torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(reps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        ev[0].record(stream)
+        for i in range(reps):
             fn()
-        e1.record(stream)
+            ev[i + 1].record(stream)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / reps
+        return percentiles([ev[i].elapsed_time(ev[i + 1]) for i in range(reps)])
 
-    ms_profile = time_fn(lambda: layer.profile(q, k, v, rows), 5)
-    ms_masks = time_fn(layer.build_masks, 5)
+    t_profile = time_fn(lambda: layer.profile(q, k, v, rows), 20)
+    t_masks = time_fn(layer.build_masks, 20)
     # the attention kernel alone on the layer's layout (the roofline's kernel),
     # and each way of doing the layout transformation, for comparison
     m = layer.masks
@@ -400,31 +473,64 @@ def main():
             g, q, k, v, kp, vp, labels_d, m[0].row_ptr, m[0].col_idx, m[1].row_ptr,
             m[1].col_idx, o)
     kp, vp = (torch.empty_like(q) for _ in range(2))
-    ms_permute_kv = time_fn(lambda: svg.svg_permute_qkv(g, None, k, v, None, kp, vp, labels_d),
-                            5)
-    ms_attn_fused = time_fn(attn_fused(kp, vp), max(3, args.steps))
-    ms_attn_gathered = time_fn(attn_fused(None, None), 3)
+    t_permute_kv = time_fn(lambda: svg.svg_permute_qkv(g, None, k, v, None, kp, vp, labels_d), 20)
+    t_attn_fused = time_fn(attn_fused(kp, vp), max(5, args.steps // 2))
+    t_attn_gathered = time_fn(attn_fused(None, None), 3)
     qp, op = (torch.empty_like(q) for _ in range(2))
-    ms_permute = time_fn(lambda: svg.svg_permute_qkv(g, q, k, v, qp, kp, vp, labels_d), 5)
-    ms_unpermute = time_fn(lambda: svg.svg_unpermute(g, op, o, labels_d), 5)
-    ms_attn_explicit = time_fn(lambda: svg.svg_sparse_attention(
-        g, q, k, v, qp, kp, vp, labels_d, m[0].row_ptr, m[0].col_idx, m[1].row_ptr,
-        m[1].col_idx, o, op), max(3, args.steps // 2))
+    t_permute = time_fn(lambda: svg.svg_permute_qkv(g, q, k, v, qp, kp, vp, labels_d), 20)
+    t_unpermute = time_fn(lambda: svg.svg_unpermute(g, op, o, labels_d), 20)
+
+    def attn_explicit():
+        svg.svg_sparse_attention(g, q, k, v, qp, kp, vp, labels_d, m[0].row_ptr, m[0].col_idx,
+                                 m[1].row_ptr, m[1].col_idx, o, op)
+    # The roofline's kernel is timed over a region of at least 2 s of back-to-back
+    # launches, long enough for the clock to settle under the power cap, and is
+    # held against the sustained bf16 peak (measured the same way); the burst
+    # fraction is reported beside it.
+    first = time_fn(attn_explicit, 2)["p50"]
+    reps_attn = max(20, int(np.ceil(2000.0 / max(first, 1e-3))))
+    attn_clocks = ClockSampler(local) if rank == 0 else None
+    t_attn_explicit = time_fn(attn_explicit, reps_attn)
+    attn_clock_info = attn_clocks.stop() if attn_clocks else None
+    attn_region_s = t_attn_explicit["mean"] * reps_attn / 1e3
+    # FP8 PV (e4m3 P and V, bf16 Q K^T): V quantised per (head, channel) from the
+    # same permuted copies, then the FP8 attention kernel on the same CSR
+    fp8 = None
+    if wl.d == 128 and wl.block_q == 128 and not args.no_fp8:
+        v8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+        v_scale = torch.empty(wl.B * wl.H * wl.d, dtype=torch.float32, device=dev)
+        t_quant = time_fn(lambda: svg.svg_quantize_v_e4m3(g, v, vp, labels_d, v8, v_scale), 20)
+        t_attn_fp8 = time_fn(lambda: svg.svg_sparse_attention_fp8pv(
+            g, q, k, qp, kp, v8, v_scale, labels_d, m[0].row_ptr, m[0].col_idx, m[1].row_ptr,
+            m[1].col_idx, o, op), max(10, args.steps))
+        # half of the algorithmic work (QK^T) at the bf16 rate, half (PV) at twice it
+        pk8 = _peaks()
+        fp8 = {"pv": "e4m3 P x e4m3 V (per-channel scales), bf16 Q K^T",
+               "quantize_v_ms": t_quant["p50"], "attention_ms": t_attn_fp8["p50"],
+               "attention_ms_pct": t_attn_fp8,
+               "attention_tflops": attn_flops / (t_attn_fp8["p50"] * 1e-3) / 1e12,
+               "speedup_vs_bf16_attention": None,
+               "mixed_peak_tflops_burst": 2.0 / (1.0 / pk8["bf16_tflops"] +
+                                                 1.0 / (2.0 * pk8["bf16_tflops"])),
+               "mixed_peak_note": "QK^T half at the measured bf16 burst peak, PV half at 2x "
+                                  "it (nominal fp8/bf16 ratio)"}
+        del v8, v_scale
     del kp, vp, qp, op
     torch.cuda.empty_cache()
-    layouts_ms = {
-        "explicit": {"permute_qkv": ms_permute, "attention": ms_attn_explicit,
-                     "unpermute": ms_unpermute,
-                     "total": ms_permute + ms_attn_explicit + ms_unpermute},
-        "fused": {"permute_kv": ms_permute_kv, "attention": ms_attn_fused,
-                  "total": ms_permute_kv + ms_attn_fused},
-        "gathered": {"attention": ms_attn_gathered, "total": ms_attn_gathered},
+    layouts = {
+        "explicit": {"permute_qkv": t_permute, "attention": t_attn_explicit,
+                     "unpermute": t_unpermute},
+        "fused": {"permute_kv": t_permute_kv, "attention": t_attn_fused},
+        "gathered": {"attention": t_attn_gathered},
     }
-    ms_attn = layouts_ms[layout]["attention"]
+    layouts_ms = {name: dict({kk: t["p50"] for kk, t in parts.items()},
+                             total=sum(t["p50"] for t in parts.values()))
+                  for name, parts in layouts.items()}
+    ms_attn = layouts[layout]["attention"]["p50"]
     ms_dense = None
     if not args.no_dense:
         od = torch.empty_like(q)
-        ms_dense = time_fn(lambda: layer.dense(q, k, v, od), 2)
+        ms_dense = time_fn(lambda: layer.dense(q, k, v, od), 3)["p50"]
         del od
     st, bits = svg.svg_get_device_status()
     if st != svg.SVG_OK:
@@ -460,27 +566,74 @@ def main():
         e2e = {"value": job_throughput(attn_flops, world, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # semantic-aware permutation (SVG2): k-means of Q and K, cluster selection,
+    # tile CSR (the plan), then gather -> attention -> scatter, on the same layer
+    svg2 = None
+    if not args.no_svg2:
+        from video_dit_spatial_b200.layer import SemanticSparseLayer
+        sl2 = SemanticSparseLayer(wl.B, wl.H, wl.N, wl.d, Cq=SVG2_CQ, Ck=SVG2_CK,
+                                  iters=SVG2_ITERS, top_p=SVG2_TOP_P, block_k=wl.block_k,
+                                  device=dev)
+        o2 = torch.empty_like(q)
+        t_plan = time_fn(lambda: sl2.plan(q, k), 5)
+        t_attend2 = time_fn(lambda: sl2.attend(q, k, v, o2), 5)
+        t_attn2 = time_fn(lambda: svg.svg2_sparse_attention(
+            wl.B * wl.H, wl.N, wl.d, wl.block_k, wl.scale, sl2.qs, sl2.ks, sl2.vs, sl2.row_ptr,
+            sl2.col_idx, sl2.os), 10)
+        rp2 = sl2.row_ptr.cpu().numpy().astype(np.int64)
+        ci2 = sl2.col_idx.cpu().numpy()[:rp2[-1]].astype(np.int64)
+        nqb2 = sl2.nqb
+        rows_in = np.tile(np.minimum(128, wl.N - np.arange(nqb2) * 128), wl.B * wl.H)
+        cols_in = np.minimum(wl.block_k, wl.N - np.arange(sl2.nkb) * wl.block_k)
+        pairs2 = int(np.sum(np.repeat(rows_in, np.diff(rp2)) * cols_in[ci2]))
+        flops2 = 4 * wl.d * pairs2
+        svg2 = {"clusters_q": SVG2_CQ, "clusters_k": SVG2_CK, "kmeans_iters": SVG2_ITERS,
+                "top_p": SVG2_TOP_P, "tile_density": float(rp2[-1]) / (wl.B * wl.H * nqb2 * sl2.nkb),
+                "plan_ms": t_plan["p50"], "attend_ms": t_attend2["p50"],
+                "attention_ms": t_attn2["p50"], "layer_ms": t_plan["p50"] + t_attend2["p50"],
+                "attention_tflops": flops2 / (t_attn2["p50"] * 1e-3) / 1e12,
+                "computed_block_tflop": flops2 / 1e12}
+        del sl2, o2
+        torch.cuda.empty_cache()
+    if fp8 is not None:
+        fp8["speedup_vs_bf16_attention"] = ms_attn / fp8["attention_ms"]
+        fp8["frac_of_mixed_peak"] = fp8["attention_tflops"] / fp8["mixed_peak_tflops_burst"]
     pk = _peaks()
     achieved = attn_flops / (ms_attn * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "sparse_attention_pair_kernel", "achieved": achieved,
-                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops_sustained"],
-                "peak_kind": f"bf16 dense, sustained, {pk['source']}",
+    sustained = attn_region_s >= 2.0
+    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    kernel_name = f"sparse_attention_pair_kernel<{wl.d},{wl.block_k}>"
+    roofline = {"bound": "tensor", "kernel": kernel_name, "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": "bf16 dense, %s, %s (kernel timed over %.1f s of back-to-back "
+                             "launches)" % ("sustained" if sustained else "burst", pk["source"],
+                                            attn_region_s),
                 "frac_of_burst_peak": achieved / pk["bf16_tflops"],
-                "traffic": _captured_traffic() if wl.name == SI.HUNYUAN.name else None,
-                "traffic_note": "ncu dram read+write of a 4-head launch, scaled by heads"}
+                "frac_of_sustained_peak": achieved / pk["bf16_tflops_sustained"],
+                "clocks": attn_clock_info,
+                "traffic": _captured_traffic(kernel_name, wl.name),
+                "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of a 4-head "
+                                "launch scaled by heads (profiles/traffic.json)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         kinds = SI.planted_head_kinds(wl)
         heads = [kinds.index(0), kinds.index(1)]
         secs, fl = oracle_sample(wl, 96, heads)
+        comps = oracle_components(wl)
+        attn_layer_s = attn_flops / (fl / secs)
         cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"fp64 oracle attention output of 96 query rows x 2 heads (one spatial, "
-                         f"one temporal) of {wl.name}, with their block-mask rows",
-               "seconds": secs,
-               # labelled extrapolation: the sample's rate over the layer's computed pairs
-               "extrapolated_layer_hours": attn_flops / (fl / secs) / 3600.0}
+                         f"one temporal) of {wl.name}, with their block-mask rows; plus "
+                         f"profiling, block masks and permutation on the samples in "
+                         f"'components'",
+               "seconds": secs + sum(c["seconds"] for c in comps.values()),
+               "components": dict(comps, attention={
+                   "seconds": secs, "sample": "96 query rows x 2 heads",
+                   "extrapolated_layer_s": attn_layer_s}),
+               # labelled extrapolation: each sample's rate over the whole layer
+               "extrapolated_layer_hours": (attn_layer_s + sum(
+                   c["extrapolated_layer_s"] for c in comps.values())) / 3600.0}
 
     if rank == 0:
         line = {
@@ -494,17 +647,20 @@ def main():
                        "n_samples": wl.n_samples,
                        "l2": "inputs larger than L2 (Q,K,V %.2f GB)" % (3 * q.numel() * 2 / 1e9),
                        "parallelism": f"independent replicas x{world}" if world > 1 else "1 GPU"},
-            "layer_ms": ms,
+            "layer_ms": ms, "layer_ms_pct": step_pct,
             "attn_ms": ms_attn, "dense_ms": ms_dense,
             "speedup_vs_dense": (ms_dense / ms_attn) if ms_dense else None,
             "layer_speedup_vs_dense": (ms_dense / ms) if ms_dense else None,
             "attn_tflops": achieved,
             "dense_tflops": (dense_flops / (ms_dense * 1e-3) / 1e12) if ms_dense else None,
             "layout": layout,
-            "kernel_ms": dict({"profile": ms_profile, "block_masks": ms_masks},
-                              **{k: t for k, t in layouts_ms[layout].items() if k != "total"}),
+            "kernel_ms": dict({"profile": t_profile["p50"], "block_masks": t_masks["p50"]},
+                              **{k: t["p50"] for k, t in layouts[layout].items()}),
+            "kernel_ms_pct": dict({"profile": t_profile, "block_masks": t_masks},
+                                  **layouts[layout]),
             "layouts_ms": layouts_ms,
             "labels_temporal": int(np.sum(labels == 1)),
+            "fp8_pv": fp8, "svg2_semantic": svg2,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": gpu_launches, "clocks": clock_info,
         }

@@ -125,3 +125,69 @@ def profile_reference(qn, kn, vn, rows, T, P, L, s, w, scale):
 
 def is_near_tie(ms, mt, tol_s, tol_t) -> bool:
     return abs(ms - mt) <= tol_s + tol_t
+
+
+# ---------------------------------------------------------------------------
+# FP8 PV: the tolerance the e4m3 rounding of P and V allows
+# ---------------------------------------------------------------------------
+# The FP8 product rounds every probability p_j = exp(s_j - m) (scaled by 2^6,
+# at a running base at most 2^2 below the row's maximum) and every V element
+# to E4M3. A rounding moves a value by at most half a grid step h: 2^-4 of it
+# for normal values, and 2^-9 / 2 = 2^-10 (in the rounded value's units) below
+# 2^-6. In the units of the exact computation that is
+#   h_p(p_j)   = max(2^-4 p_j, 2^-10 * 2^-6)       (a lower running base only
+#                                                    shrinks the subnormal part)
+#   h_v(v_jc)  = max(2^-4 |v_jc|, 2^-10 * scale_c)
+# and an output element O_ic = sum_j w_j v_jc (w = p / l, l = sum p in fp32,
+# not rounded) moves by sum_j (w_j dv_jc + dp_j v_jc / l). Taking each rounding
+# error as an independent zero-mean variable of variance at most h^2 (the
+# worst case of any distribution on [-h, h]) gives
+#   sigma_ic^2 = sum_j w_j^2 h_v(v_jc)^2 + sum_j (h_p(p_j) / l)^2 v_jc^2,
+# and the element-wise bar |O - O*| <= 6 sigma_ic + 2^-8 |O*_ic| (the bf16
+# rounding of the output) + 1e-6.
+def fp8_reference(qn, kn, vn, label, T, P, L, s, w, bq, bk, scale, rows):
+    """(O* [r, d], tol [r, d]) at frame-major `rows` of one head: the oracle's
+    block-sparse attention (oracle.layer_rows) and the FP8 tolerance above."""
+    N = qn.shape[0]
+    want, _ = O.layer_rows(qn, kn, vn, label, T, P, L, s, w, bq, bk, scale, rows=rows)
+    kind = O.MASK_TEMPORAL if label == O.HEAD_TEMPORAL else O.MASK_SPATIAL
+    rows = np.asarray(rows, dtype=np.int64)
+    if kind == O.MASK_TEMPORAL:
+        pi = O.permutation(T, P, L)
+        lrows = pi[rows]
+        ql, kl, vl = (O.permute(x, T, P, L) for x in (qn, kn, vn))
+    else:
+        lrows, ql, kl, vl = rows, qn, kn, vn
+    needed = np.unique(lrows // bq)
+    bm = np.zeros((O.n_blocks(N, bq), O.n_blocks(N, bk)), dtype=bool)
+    bm[needed] = O.block_mask_rows(kind, needed, T, P, L, s, w, bq, bk)
+    _, vscale = O.quantize_v_e4m3(vl)
+    sc = vscale.astype(np.float64)
+    xv = np.abs(vl) / np.where(sc > 0, sc, 1.0)[None, :]
+    hv2 = np.where(xv >= 2.0 ** -6, 2.0 ** -4 * np.abs(vl), 2.0 ** -10 * sc[None, :]) ** 2
+    v2 = vl * vl
+    tol = np.zeros((rows.size, vn.shape[1]))
+    for c0 in range(0, rows.size, _CHUNK):
+        rr = lrows[c0:c0 + _CHUNK]
+        wts = O.attention_weights_rows(ql, kl, rr, O.block_allowed_fn(bm, bq, bk, N), scale)
+        wmax = wts.max(axis=1, keepdims=True)  # = 1 / l
+        p = wts / wmax
+        hp = np.maximum(2.0 ** -4 * p, 2.0 ** -16)
+        hp = np.where(wts > 0, hp, 0.0)  # keys outside the computed blocks take no part
+        var = (wts * wts) @ hv2 + ((hp * wmax) ** 2) @ v2
+        tol[c0:c0 + rr.size] = 6.0 * np.sqrt(var)
+    tol += 2.0 ** -8 * np.abs(want) + 1e-6
+    return want, tol
+
+
+def assert_within(got, want, tol, what):
+    """Element-wise |got - want| <= tol; prints the FP8 PARITY line."""
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - want)
+    norm = float(np.sqrt(np.sum(want * want)))
+    rel = float(np.sqrt(np.sum(err * err)) / norm) if norm > 0 else 0.0
+    ratio = float(np.max(err / tol))
+    print(f"PARITY-FP8 {what}: max_abs {err.max():.3e} mean_abs {err.mean():.3e} "
+          f"rel_l2 {rel:.3e} max err/tol {ratio:.3f}")
+    assert ratio <= 1.0, f"{what}: error exceeds the e4m3 bound by {ratio:.3f}x"
+    return float(err.max()), float(err.mean()), rel
