@@ -39,6 +39,7 @@ DEFAULT_WORKLOAD = SI.HUNYUAN.name
 # the semantic-aware (SVG2) measurement: clusters of queries and keys, Lloyd
 # iterations and the kept share of the centroid attention
 SVG2_CQ, SVG2_CK, SVG2_ITERS, SVG2_TOP_P = 256, 256, 10, 0.9
+SVG2_EAR_TAU = 0.01  # SVG-EAR: route skipped cluster pairs whose estimated error exceeds it
 
 
 def _peaks():
@@ -334,6 +335,24 @@ def run_capture(args, wl):
         "profile": lambda: fu.profile(q, k, v, rows),
         "permute": lambda: svg.svg_permute_qkv(g, q, k, v, ex.qp, ex.kp, ex.vp, ex.labels),
     }
+    if args.capture in ("kmeans", "ear"):
+        from video_dit_spatial_b200.layer import SemanticSparseLayer
+        sl2 = SemanticSparseLayer(wl.B, wl.H, wl.N, wl.d, Cq=SVG2_CQ, Ck=SVG2_CK, iters=1,
+                                  top_p=SVG2_TOP_P, block_k=wl.block_k,
+                                  ear_tau=SVG2_EAR_TAU if args.capture == "ear" else None)
+        sl2.plan(q, k, v)
+        sl2.attend(q, k, v, o)
+        BH = wl.B * wl.H
+        if args.capture == "kmeans":
+            # one assignment + sort + update round of the query clustering
+            c_out = torch.empty_like(sl2.cq)
+            fns["kmeans"] = lambda: svg.svg2_kmeans_step(
+                BH, wl.N, wl.d, SVG2_CQ, q, sl2.cq, c_out, sl2.assign_q, sl2.order_q,
+                sl2.offsets_q, sl2.workspace)
+        else:
+            fns["ear"] = lambda: svg.svg2_ear_compensate(
+                BH, wl.N, wl.d, SVG2_CK, wl.block_k, wl.scale, sl2.qs, sl2.ck, sl2.vbar,
+                sl2.offsets_k, sl2.row_ptr, sl2.col_idx, sl2.os, sl2.lse, sl2.ear_ws)
     if args.capture == "attention_fp8":
         v8 = torch.empty(q.shape, dtype=torch.uint8, device="cuda")
         v_scale = torch.empty(wl.B * wl.H * wl.d, dtype=torch.float32, device="cuda")
@@ -370,7 +389,8 @@ def main():
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-svg2", action="store_true")
     ap.add_argument("--capture", choices=["attention", "attention_fused", "attention_gathered",
-                                          "attention_fp8", "profile", "permute"],
+                                          "attention_fp8", "profile", "permute", "kmeans",
+                                          "ear"],
                     help="small case for an ncu capture: run one kernel 3 times on the "
                          "workload with --heads heads, print per-launch ms, no JSON line")
     ap.add_argument("--heads", type=int, default=4)
@@ -593,7 +613,24 @@ def main():
                 "attention_ms": t_attn2["p50"], "layer_ms": t_plan["p50"] + t_attend2["p50"],
                 "attention_tflops": flops2 / (t_attn2["p50"] * 1e-3) / 1e12,
                 "computed_block_tflop": flops2 / 1e12}
-        del sl2, o2
+        del sl2
+        torch.cuda.empty_cache()
+        # SVG-EAR on the same layer: routing, then compensation of what is left out
+        se = SemanticSparseLayer(wl.B, wl.H, wl.N, wl.d, Cq=SVG2_CQ, Ck=SVG2_CK,
+                                 iters=SVG2_ITERS, top_p=SVG2_TOP_P, block_k=wl.block_k,
+                                 ear_tau=SVG2_EAR_TAU, device=dev)
+        t_plan_e = time_fn(lambda: se.plan(q, k, v), 5)
+        t_attend_e = time_fn(lambda: se.attend(q, k, v, o2), 5)
+        t_comp = time_fn(lambda: svg.svg2_ear_compensate(
+            wl.B * wl.H, wl.N, wl.d, SVG2_CK, wl.block_k, wl.scale, se.qs, se.ck, se.vbar,
+            se.offsets_k, se.row_ptr, se.col_idx, se.os, se.lse, se.ear_ws), 10)
+        rpe = se.row_ptr.cpu().numpy().astype(np.int64)
+        svg2["ear"] = {"tau": SVG2_EAR_TAU,
+                       "tile_density": float(rpe[-1]) / (wl.B * wl.H * se.nqb * se.nkb),
+                       "plan_ms": t_plan_e["p50"], "attend_ms": t_attend_e["p50"],
+                       "compensate_ms": t_comp["p50"],
+                       "layer_ms": t_plan_e["p50"] + t_attend_e["p50"]}
+        del se, o2
         torch.cuda.empty_cache()
     if fp8 is not None:
         fp8["speedup_vs_bf16_attention"] = ms_attn / fp8["attention_ms"]

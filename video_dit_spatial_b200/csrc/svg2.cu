@@ -186,7 +186,9 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     for (int j = 0; j < n; ++j) {
       const int st = j & 1;
-      if (!mbar_wait(&bar->s_full[st], (j >> 1) & 1, abort_flag, p.status)) break;
+      // warp-uniform: the tensor-memory loads below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[st], (j >> 1) & 1, abort_flag, p.status)))
+        break;
       tc_fence_after();
       float best = INFINITY;
       int best_c = 0;
@@ -839,8 +841,10 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
       }
     }
   } else {
+    // Every tcgen05.ld / st below is warp-collective: the branches around them
+    // are warp-uniform, and only the global loads and stores depend on the row.
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    bool ok = mbar_wait(&bar->s_full, 0, abort_flag, p.status);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&bar->s_full, 0, abort_flag, p.status));
     float m = -INFINITY, den = 0.0f;
     if (ok) {
       tc_fence_after();
@@ -899,13 +903,15 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
     }
     tc_fence_before();
     mbar_arrive(&bar->p_full);
-    if (ok) ok = mbar_wait(&bar->o_full, 0, abort_flag, p.status);
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->o_full, 0, abort_flag, p.status));
     tc_fence_after();
-    // merge with the sparse output of this row
+    // merge with the sparse output of this row (rows past N only take part in
+    // the warp's tensor-memory loads)
     const int qrow = r * 128 + tid;
-    if (__all_sync(0xffffffffu, ok) && qrow < p.N) {
-      const size_t ro = static_cast<size_t>(bh) * p.N + qrow;
-      const float lse2 = p.lse[ro] * 1.4426950408889634f;
+    const bool row_ok = qrow < p.N;
+    if (ok) {
+      const size_t ro = static_cast<size_t>(bh) * p.N + (row_ok ? qrow : 0);
+      const float lse2 = row_ok ? p.lse[ro] * 1.4426950408889634f : -INFINITY;
       const float M = fmaxf(lse2, m);
       const float a = lse2 == -INFINITY ? 0.0f : fast_exp2(lse2 - M);
       const float c = m == -INFINITY ? 0.0f : fast_exp2(m - M);
@@ -918,6 +924,7 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
         tmem_ld_32x32b_x32(lane_base + Cf::kColO + ch * 32, o);
         tmem_ld_wait();
         reg_fence(o);
+        if (!row_ok) continue;
         uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
         uint32_t pk[16];
 #pragma unroll
