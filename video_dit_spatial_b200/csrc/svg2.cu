@@ -355,43 +355,93 @@ __global__ void sort_rank_kernel(const int32_t* __restrict__ assign, const int32
 }
 
 // ------------------------------------------------------------ update
-// One warp per (bh, c): the mean of the members (sorted order) in fp32.
+// Members of a cluster, summed by one CTA of kSumWarps warps: warp w takes the
+// w-th of kSumWarps equal runs of the cluster's sorted positions and adds its
+// rows in order (kBatch row loads in flight), lane l holding channels
+// [D/32 * l, D/32 * (l+1)); the warps' partial sums are then added in warp
+// order. The order of every addition is fixed: the result is deterministic.
+constexpr int kSumWarps = 4;
+constexpr int kBatch = 8;
+
 template <int D>
-__global__ void kmeans_update_kernel(const svg_bf16* __restrict__ x, const int32_t* __restrict__ order,
-                                     const int32_t* __restrict__ offsets, int32_t N, int32_t C,
-                                     int32_t rows, const float* __restrict__ c_in,
-                                     float* __restrict__ c_out) {
-  constexpr int kPer = D / 32;  // channels per lane
-  const int gw = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (gw >= rows) return;
-  const int bh = gw / C, c = gw - bh * C;
+__device__ __forceinline__ void load_row_slice(const svg_bf16* __restrict__ x, size_t row,
+                                               int lane, float (&out)[D / 32]) {
+  const svg_bf16* src = x + row * D + lane * (D / 32);
+  if constexpr (D / 32 == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(src);
+    out[0] = __uint_as_float(u.x << 16);
+    out[1] = __uint_as_float(u.x & 0xffff0000u);
+    out[2] = __uint_as_float(u.y << 16);
+    out[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+    out[0] = __uint_as_float(u << 16);
+    out[1] = __uint_as_float(u & 0xffff0000u);
+  }
+}
+
+// sum[i] += the rows at sorted positions [q0, q1) of head bh, in order (or,
+// with center, their squared deviations from it)
+template <int D>
+__device__ __forceinline__ void sum_rows(const svg_bf16* __restrict__ x,
+                                         const int32_t* __restrict__ order, int32_t N, int bh,
+                                         int q0, int q1, int lane, float (&sum)[D / 32],
+                                         const float* center) {
+  constexpr int kPer = D / 32;
+  const int32_t* ord = order + static_cast<size_t>(bh) * N;
+  for (int base = q0; base < q1; base += kBatch) {
+    float v[kBatch][kPer];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (base + u < q1)
+        load_row_slice<D>(x, static_cast<size_t>(bh) * N + __ldg(ord + base + u), lane, v[u]);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (base + u >= q1) break;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        if (center == nullptr) {
+          sum[i] += v[u][i];
+        } else {
+          const float dv = v[u][i] - center[i];
+          sum[i] = fmaf(dv, dv, sum[i]);
+        }
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(32 * kSumWarps)
+    kmeans_update_kernel(const svg_bf16* __restrict__ x, const int32_t* __restrict__ order,
+                         const int32_t* __restrict__ offsets, int32_t N, int32_t C,
+                         const float* __restrict__ c_in, float* __restrict__ c_out) {
+  constexpr int kPer = D / 32;
+  __shared__ float part[kSumWarps][D];
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
-  const int p0 = off[c], p1 = off[c + 1];
+  const int p0 = off[c], p1 = off[c + 1], cnt = p1 - p0;
+  const int q0 = p0 + static_cast<int>(static_cast<long long>(cnt) * w / kSumWarps);
+  const int q1 = p0 + static_cast<int>(static_cast<long long>(cnt) * (w + 1) / kSumWarps);
   float acc[kPer];
 #pragma unroll
   for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
-  for (int pos = p0; pos < p1; ++pos) {
-    const int r = order[static_cast<size_t>(bh) * N + pos];
-    const svg_bf16* src = x + (static_cast<size_t>(bh) * N + r) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(src);
-      acc[0] += __uint_as_float(u.x << 16);
-      acc[1] += __uint_as_float(u.x & 0xffff0000u);
-      acc[2] += __uint_as_float(u.y << 16);
-      acc[3] += __uint_as_float(u.y & 0xffff0000u);
-    } else {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
-      acc[0] += __uint_as_float(u << 16);
-      acc[1] += __uint_as_float(u & 0xffff0000u);
+  sum_rows<D>(x, order, N, bh, q0, q1, lane, acc, nullptr);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) part[w][lane * kPer + i] = acc[i];
+  __syncthreads();
+  if (w == 0) {
+    float* dst = c_out + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+    const float* prev = c_in + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      float tot = 0.0f;
+#pragma unroll
+      for (int ww = 0; ww < kSumWarps; ++ww) tot += part[ww][lane * kPer + i];
+      dst[i] = cnt > 0 ? __fdiv_rn(tot, static_cast<float>(cnt)) : prev[i];
     }
   }
-  float* dst = c_out + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
-  const float* prev = c_in + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
-  const int cnt = p1 - p0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i)
-    dst[i] = cnt > 0 ? __fdiv_rn(acc[i], static_cast<float>(cnt)) : prev[i];
 }
 
 // ------------------------------------------------------------ selection
@@ -612,63 +662,67 @@ __global__ void permute_rows_kernel(const svg_bf16* __restrict__ x, const int32_
 }
 
 // ------------------------------------------------------------ SVG-EAR
-// Per key cluster (one warp per (bh, b)), over its members in sorted order:
-// vbar = the fp32 mean value, disp = sqrt(mean over members and channels of
-// (v - vbar)^2); an empty cluster gets zeros.
+// Per key cluster (one CTA of kSumWarps warps per (bh, b), the update kernel's
+// fixed split and order), over its members in sorted order: vbar = the fp32
+// mean value, disp = sqrt(mean over members and channels of (v - vbar)^2); an
+// empty cluster gets zeros.
 template <int D>
-__global__ void cluster_stats_kernel(const svg_bf16* __restrict__ v, const int32_t* __restrict__ order,
-                                     const int32_t* __restrict__ offsets, int32_t N, int32_t C,
-                                     int32_t rows, float* __restrict__ vbar,
-                                     float* __restrict__ disp) {
+__global__ void __launch_bounds__(32 * kSumWarps)
+    cluster_stats_kernel(const svg_bf16* __restrict__ v, const int32_t* __restrict__ order,
+                         const int32_t* __restrict__ offsets, int32_t N, int32_t C,
+                         float* __restrict__ vbar, float* __restrict__ disp) {
   constexpr int kPer = D / 32;
-  const int gw = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (gw >= rows) return;
-  const int bh = gw / C, c = gw - bh * C;
+  __shared__ float part[kSumWarps][D];
+  __shared__ float mean_s[D];
+  __shared__ float sq_s[kSumWarps];
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
-  const int p0 = off[c], p1 = off[c + 1];
-  auto load = [&](int pos, float (&x)[kPer]) {
-    const int r = order[static_cast<size_t>(bh) * N + pos];
-    const svg_bf16* src = v + (static_cast<size_t>(bh) * N + r) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(src);
-      x[0] = __uint_as_float(u.x << 16);
-      x[1] = __uint_as_float(u.x & 0xffff0000u);
-      x[2] = __uint_as_float(u.y << 16);
-      x[3] = __uint_as_float(u.y & 0xffff0000u);
-    } else {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
-      x[0] = __uint_as_float(u << 16);
-      x[1] = __uint_as_float(u & 0xffff0000u);
+  const int p0 = off[c], p1 = off[c + 1], cnt = p1 - p0;
+  const int q0 = p0 + static_cast<int>(static_cast<long long>(cnt) * w / kSumWarps);
+  const int q1 = p0 + static_cast<int>(static_cast<long long>(cnt) * (w + 1) / kSumWarps);
+  float acc[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+  sum_rows<D>(v, order, N, bh, q0, q1, lane, acc, nullptr);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) part[w][lane * kPer + i] = acc[i];
+  __syncthreads();
+  if (w == 0) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      float tot = 0.0f;
+#pragma unroll
+      for (int ww = 0; ww < kSumWarps; ++ww) tot += part[ww][lane * kPer + i];
+      mean_s[lane * kPer + i] = cnt > 0 ? __fdiv_rn(tot, static_cast<float>(cnt)) : 0.0f;
     }
-  };
-  float mean[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) mean[i] = 0.0f;
-  for (int pos = p0; pos < p1; ++pos) {
-    float x[kPer];
-    load(pos, x);
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) mean[i] += x[i];
   }
-  const int cnt = p1 - p0;
+  __syncthreads();
+  float center[kPer], sq[kPer];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) mean[i] = cnt > 0 ? __fdiv_rn(mean[i], static_cast<float>(cnt)) : 0.0f;
-  float sq = 0.0f;
-  for (int pos = p0; pos < p1; ++pos) {
-    float x[kPer];
-    load(pos, x);
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) sq = fmaf(x[i] - mean[i], x[i] - mean[i], sq);
+  for (int i = 0; i < kPer; ++i) {
+    center[i] = mean_s[lane * kPer + i];
+    sq[i] = 0.0f;
   }
-  float tot = 0.0f;
-  for (int l = 0; l < 32; ++l) tot += __shfl_sync(0xffffffffu, sq, l);
-  float* dst = vbar + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+  sum_rows<D>(v, order, N, bh, q0, q1, lane, sq, center);
+  float lane_sq = 0.0f;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) dst[i] = mean[i];
-  if (lane == 0)
-    disp[static_cast<size_t>(bh) * C + c] =
-        cnt > 0 ? sqrtf(__fdiv_rn(tot, static_cast<float>(cnt) * D)) : 0.0f;
+  for (int i = 0; i < kPer; ++i) lane_sq += sq[i];
+  float wsum = 0.0f;
+  for (int l = 0; l < 32; ++l) wsum += __shfl_sync(0xffffffffu, lane_sq, l);
+  if (lane == 0) sq_s[w] = wsum;
+  __syncthreads();
+  if (w == 0) {
+    float* dst = vbar + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) dst[i] = mean_s[lane * kPer + i];
+    if (lane == 0) {
+      float tot = 0.0f;
+      for (int ww = 0; ww < kSumWarps; ++ww) tot += sq_s[ww];
+      disp[static_cast<size_t>(bh) * C + c] =
+          cnt > 0 ? sqrtf(__fdiv_rn(tot, static_cast<float>(cnt) * D)) : 0.0f;
+    }
+  }
 }
 
 // fp32 [rows, D] -> bf16 [rows, D] (round to nearest even)
@@ -1054,13 +1108,13 @@ cudaError_t launch_cluster_sort(int32_t BH, int32_t N, int32_t C, const int32_t*
 cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
                                  const int32_t* order, const int32_t* offsets, const float* c_in,
                                  float* c_out, cudaStream_t stream) {
-  const int rows = BH * C;
+  const dim3 grid(static_cast<unsigned>(C), static_cast<unsigned>(BH));
   if (D == 128)
-    kmeans_update_kernel<128><<<(rows + 7) / 8, 256, 0, stream>>>(x, order, offsets, N, C, rows,
-                                                                 c_in, c_out);
+    kmeans_update_kernel<128><<<grid, 32 * kSumWarps, 0, stream>>>(x, order, offsets, N, C, c_in,
+                                                                   c_out);
   else
-    kmeans_update_kernel<64><<<(rows + 7) / 8, 256, 0, stream>>>(x, order, offsets, N, C, rows,
-                                                                c_in, c_out);
+    kmeans_update_kernel<64><<<grid, 32 * kSumWarps, 0, stream>>>(x, order, offsets, N, C, c_in,
+                                                                  c_out);
   return cudaGetLastError();
 }
 
@@ -1154,13 +1208,13 @@ namespace svg {
 cudaError_t launch_cluster_stats(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* v,
                                  const int32_t* order, const int32_t* offsets, float* vbar,
                                  float* disp, cudaStream_t stream) {
-  const int rows = BH * C;
+  const dim3 grid(static_cast<unsigned>(C), static_cast<unsigned>(BH));
   if (D == 128)
-    cluster_stats_kernel<128><<<(rows + 7) / 8, 256, 0, stream>>>(v, order, offsets, N, C, rows,
-                                                                 vbar, disp);
+    cluster_stats_kernel<128><<<grid, 32 * kSumWarps, 0, stream>>>(v, order, offsets, N, C, vbar,
+                                                                   disp);
   else
-    cluster_stats_kernel<64><<<(rows + 7) / 8, 256, 0, stream>>>(v, order, offsets, N, C, rows,
-                                                                vbar, disp);
+    cluster_stats_kernel<64><<<grid, 32 * kSumWarps, 0, stream>>>(v, order, offsets, N, C, vbar,
+                                                                  disp);
   return cudaGetLastError();
 }
 
