@@ -612,6 +612,8 @@ def main():
                 "plan_ms": t_plan["p50"], "attend_ms": t_attend2["p50"],
                 "attention_ms": t_attn2["p50"], "layer_ms": t_plan["p50"] + t_attend2["p50"],
                 "attention_tflops": flops2 / (t_attn2["p50"] * 1e-3) / 1e12,
+                "attention_frac_of_burst_peak": flops2 / (t_attn2["p50"] * 1e-3) / 1e12 /
+                _peaks()["bf16_tflops"],
                 "computed_block_tflop": flops2 / 1e12}
         del sl2
         torch.cuda.empty_cache()
