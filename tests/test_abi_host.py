@@ -208,3 +208,71 @@ def test_python_binding_rejects_host_tensors():
     with pytest.raises(ValueError, match="device buffers"):
         m._ptr(x.transpose(2, 3))
     assert m._ptr(None) is None and m._ptr(1234) == 1234
+
+
+def test_fp8_and_svg2_arguments_are_rejected_before_launch(svg):
+    """Host-side validation of the FP8, SVG2 and SVG-EAR entry points: every
+    case below is refused before any device call (no GPU needed)."""
+    lib = svg.load()
+    g64 = _geom(svg, d=64, bq=128, bk=128)
+    g128 = _geom(svg, d=128, bq=128, bk=128)
+    gq64 = _geom(svg, d=128, bq=64, bk=128)
+    # FP8: d = 128 only; block_q = 128 only; labels need vp; misaligned codes
+    assert lib.svg_quantize_v_e4m3(ctypes.byref(g64), 256, None, None, 256, 256, None) == \
+        svg.SVG_ERR_UNSUPPORTED
+    assert lib.svg_quantize_v_e4m3(ctypes.byref(g128), 256, None, 256, 256, 256, None) == \
+        svg.SVG_ERR_INVALID_ARG
+    assert lib.svg_quantize_v_e4m3(ctypes.byref(g128), 256, None, None, 264, 256, None) == \
+        svg.SVG_ERR_INVALID_ARG
+    fa = lib.svg_sparse_attention_fp8pv
+    assert fa(ctypes.byref(gq64), 256, 256, None, None, 256, 256, None, 256, 256, None, None,
+              256, None, None, None) == svg.SVG_ERR_UNSUPPORTED
+    assert fa(ctypes.byref(g128), 256, 256, 256, None, 256, 256, None, 256, 256, None, None,
+              256, None, None, None) == svg.SVG_ERR_INVALID_ARG  # qp without kp/op
+    # SVG2 k-means: C a multiple of 16 in [16, 256], d 64 or 128
+    ws = ctypes.c_size_t()
+    assert lib.svg2_kmeans_workspace_bytes(2, 1000, 128, 17, ctypes.byref(ws)) == \
+        svg.SVG_ERR_UNSUPPORTED
+    assert lib.svg2_kmeans_workspace_bytes(2, 1000, 128, 272, ctypes.byref(ws)) == \
+        svg.SVG_ERR_UNSUPPORTED
+    assert lib.svg2_kmeans_workspace_bytes(2, 1000, 96, 32, ctypes.byref(ws)) == \
+        svg.SVG_ERR_UNSUPPORTED
+    assert lib.svg2_kmeans_workspace_bytes(2, 1000, 128, 32, ctypes.byref(ws)) == svg.SVG_OK
+    need = ws.value
+    assert lib.svg2_kmeans(2, 1000, 128, 32, 3, 256, 256, 256, 256, 256, 256, need - 1,
+                           None) == svg.SVG_ERR_CAPACITY
+    assert lib.svg2_kmeans(2, 1000, 128, 32, 3, 256, 256, 256, 256, 256, 264, need,
+                           None) == svg.SVG_ERR_INVALID_ARG  # workspace not 256-aligned
+    assert lib.svg2_kmeans_step(2, 1000, 128, 32, 256, 512, 512, 256, 256, 256, 256, need,
+                                None) == svg.SVG_ERR_INVALID_ARG  # in place
+    # selection: Ck <= 1024, 0 < top_p <= 1, tau >= 0 when routing
+    sel = lib.svg2_select_clusters
+    assert sel(1, 128, 8, 1025, ctypes.c_float(0.1), ctypes.c_float(0.9), 256, 256, 256, None,
+               ctypes.c_float(0.0), 256, None) == svg.SVG_ERR_INVALID_ARG
+    assert sel(1, 128, 8, 64, ctypes.c_float(0.1), ctypes.c_float(1.5), 256, 256, 256, None,
+               ctypes.c_float(0.0), 256, None) == svg.SVG_ERR_INVALID_ARG
+    assert sel(1, 128, 8, 64, ctypes.c_float(0.1), ctypes.c_float(0.9), 256, 256, 256, 256,
+               ctypes.c_float(-1.0), 256, None) == svg.SVG_ERR_INVALID_ARG
+    # tile CSR: blocks 64 or 128; at most 4096 key tiles
+    csr = lib.svg2_build_tile_csr
+    assert csr(1, 1000, 8, 8, 96, 128, 256, 256, 256, 256, 256, 100, 256, None) == \
+        svg.SVG_ERR_UNSUPPORTED
+    assert csr(1, 4097 * 64, 8, 8, 128, 64, 256, 256, 256, 256, 256, 100, 256, None) == \
+        svg.SVG_ERR_UNSUPPORTED
+    # row permutation: overlapping buffers, d
+    assert lib.svg2_gather_rows(1, 100, 128, 4096, 256, 4096 + 256, None) == \
+        svg.SVG_ERR_INVALID_ARG
+    assert lib.svg2_scatter_rows(1, 100, 96, 4096, 256, 1 << 20, None) == \
+        svg.SVG_ERR_UNSUPPORTED
+    # attention on sorted layouts: d and block_k
+    assert lib.svg2_sparse_attention(1, 1000, 96, 128, ctypes.c_float(0.1), *([256] * 6), None,
+                                     None) == svg.SVG_ERR_UNSUPPORTED
+    # SVG-EAR: Ck a multiple of 16 in [16, 256]; workspace size
+    ews = ctypes.c_size_t()
+    assert lib.svg2_ear_workspace_bytes(2, 128, 64, ctypes.byref(ews)) == svg.SVG_OK
+    assert ews.value >= 2 * 64 * 128 * 2 * 2
+    comp = lib.svg2_ear_compensate
+    assert comp(2, 1000, 128, 40, 128, ctypes.c_float(0.1), *([256] * 9), ews.value, None) == \
+        svg.SVG_ERR_UNSUPPORTED
+    assert comp(2, 1000, 128, 64, 128, ctypes.c_float(0.1), *([256] * 9), ews.value - 1,
+                None) == svg.SVG_ERR_CAPACITY
