@@ -645,10 +645,9 @@ __global__ void permute_rows_kernel(const svg_bf16* __restrict__ x, const int32_
   const int64_t total = static_cast<int64_t>(BH) * N * vec;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t rowi = i / vec;
+    const int64_t rowi = i / vec;  // bh * N + sorted position
     const int v = static_cast<int>(i - rowi * vec);
     const int64_t bh = rowi / N;
-    const int pos = static_cast<int>(rowi - bh * N);
     const int r = order[rowi];
     if (r < 0 || r >= N) {
       atomicOr(status, kDevErrBounds);
@@ -657,7 +656,6 @@ __global__ void permute_rows_kernel(const svg_bf16* __restrict__ x, const int32_
     const int64_t src = kScatter ? rowi : bh * N + r;
     const int64_t dst = kScatter ? bh * N + r : rowi;
     reinterpret_cast<uint4*>(y + dst * D)[v] = reinterpret_cast<const uint4*>(x + src * D)[v];
-    (void)pos;
   }
 }
 
