@@ -507,7 +507,9 @@ def main():
     # launches, long enough for the clock to settle under the power cap, and is
     # held against the sustained bf16 peak (measured the same way); the burst
     # fraction is reported beside it.
-    first = time_fn(attn_explicit, 2)["p50"]
+    # the three layouts compared under the same conditions (the same short run)
+    t_attn_explicit_short = time_fn(attn_explicit, max(5, args.steps // 2))
+    first = t_attn_explicit_short["p50"]
     reps_attn = max(20, int(np.ceil(2000.0 / max(first, 1e-3))))
     attn_clocks = ClockSampler(local) if rank == 0 else None
     t_attn_explicit = time_fn(attn_explicit, reps_attn)
@@ -538,7 +540,7 @@ def main():
     del kp, vp, qp, op
     torch.cuda.empty_cache()
     layouts = {
-        "explicit": {"permute_qkv": t_permute, "attention": t_attn_explicit,
+        "explicit": {"permute_qkv": t_permute, "attention": t_attn_explicit_short,
                      "unpermute": t_unpermute},
         "fused": {"permute_kv": t_permute_kv, "attention": t_attn_fused},
         "gathered": {"attention": t_attn_gathered},
@@ -546,6 +548,12 @@ def main():
     layouts_ms = {name: dict({kk: t["p50"] for kk, t in parts.items()},
                              total=sum(t["p50"] for t in parts.values()))
                   for name, parts in layouts.items()}
+    # the roofline's kernel: the layer's layout, from the long region when that is
+    # the explicit layout (the default)
+    if layout == "explicit":
+        layouts[layout]["attention"] = t_attn_explicit
+    else:
+        attn_region_s = 0.0
     ms_attn = layouts[layout]["attention"]["p50"]
     ms_dense = None
     if not args.no_dense:
