@@ -346,9 +346,10 @@ svg_status svg2_kmeans_workspace_bytes(int32_t BH, int32_t N, int32_t d, int32_t
  *               the centroids rounded to bf16 for the distance (a tcgen05
  *               product X C^T, fp32 accumulation), ties to the smaller index;
  *   update      each centroid = the fp32 mean of its members (an empty
- *               cluster keeps its centroid), summed in a fixed order: four
- *               consecutive runs of the cluster's sorted members, each in
- *               order, then the four partial sums in run order.
+ *               cluster keeps its centroid), summed in a fixed order: the
+ *               sorted positions are cut into chunks of 256; the members in
+ *               each chunk are added in order, then the chunks' sums in
+ *               chunk order.
  * Outputs the final centroids, the last iteration's assignment (the one the
  * centroids are the means of) and its stable cluster order: order[bh, pos] =
  * row at sorted position pos (rows sorted by cluster, ties by row index),
@@ -394,7 +395,9 @@ svg_status svg2_select_clusters(int32_t BH, int32_t d, int32_t Cq, int32_t Ck, f
                                 uint32_t* sel, svg_stream_t stream);
 
 /* svg2_cluster_value_stats -- SVG-EAR statistics of every key cluster, over
- * its members (summed in the fixed order of svg2_kmeans' update): vbar[bh, b] = the fp32 mean of their values,
+ * its members (summed in a fixed order: four consecutive runs of the
+ * cluster's sorted members, each in order, then the four run sums in order):
+ * vbar[bh, b] = the fp32 mean of their values,
  * disp[bh, b] = sqrt(mean over members and channels of (v - vbar)^2); an
  * empty cluster gets zeros. v bf16 [BH, N, d] (original order), order_k and
  * offsets_k from svg2_kmeans of the keys; vbar fp32 [BH, Ck, d] (16-byte

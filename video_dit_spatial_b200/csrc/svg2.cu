@@ -26,7 +26,8 @@
 //                          in tensor memory, then a per-row argmin of
 //                          |c|^2 - 2 x.c (one softmax-style warpgroup)
 //   sort_hist / sort_scan / sort_rank   stable counting sort by cluster
-//   kmeans_update_kernel   per cluster, the members' mean in sorted order
+//   kmeans_chunk_sum / kmeans_mean kernels   the members' means: run sums
+//                          per chunk of sorted positions, then per cluster
 //   select_kernel          the top-p key clusters of each query cluster
 //   tile_count / tile_fill kernels      per-head CSR of the tile pairs
 //   gather / scatter rows  the permutation of Q, K, V and of the output
@@ -38,14 +39,17 @@ namespace svg {
 namespace {
 
 // ------------------------------------------------------------ assignment
-constexpr int kAsgThreads = 192;  // warps 0-3 argmin, 4 producer, 5 MMA
-constexpr int kAsgProducer = 4;
-constexpr int kAsgMma = 5;
+// warps 0-7 argmin (warpgroup g takes the row tiles j with j % 2 == g, in
+// tensor-memory buffer g), warp 8 TMA producer, warp 9 MMA issuer
+constexpr int kAsgThreads = 320;
+constexpr int kAsgProducer = 8;
+constexpr int kAsgMma = 9;
+constexpr int kAsgXStages = 4;
 constexpr int kMaxC = 256;  // centroids per assignment launch (one MMA N)
 
 struct AsgBarriers {
   uint64_t c_full;
-  uint64_t x_full[2], x_empty[2];
+  uint64_t x_full[kAsgXStages], x_empty[kAsgXStages];
   uint64_t s_full[2], s_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -61,7 +65,7 @@ struct AsgCfg {
   static constexpr int kCBytes = kPanels * kCPanel;
   static constexpr int kOffC = 0;
   static constexpr int kOffX = kOffC + kCBytes;
-  static constexpr int kOffNorm = kOffX + 2 * kXBytes;
+  static constexpr int kOffNorm = kOffX + kAsgXStages * kXBytes;
   static constexpr int kOffBar = kOffNorm + kMaxC * 4;
   static constexpr int kBarBytes = (static_cast<int>(sizeof(AsgBarriers)) + 127) / 128 * 128;
   static constexpr int kUsed = kOffBar + kBarBytes + 1024;
@@ -109,9 +113,11 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
   }
   if (tid == 32) {
     mbar_init(&bar->c_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kAsgXStages; ++s) {
       mbar_init(&bar->x_full[s], 1);
       mbar_init(&bar->x_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->s_full[s], 1);
       mbar_init(&bar->s_empty[s], 128);
     }
@@ -132,8 +138,9 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         tma_load_3d(sC + pn * Cf::kCPanel, &p.tm_c, &bar->c_full, pn * 64, 0, bh);
       int issued = 0;
       for (int j = 0; j < n; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(&bar->x_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        const int st = j % kAsgXStages;
+        if (!mbar_wait(&bar->x_empty[st], ((j / kAsgXStages) & 1) ^ 1, abort_flag, p.status))
+          break;
         mbar_arrive_expect_tx(&bar->x_full[st], Cf::kXBytes);
         for (int pn = 0; pn < Cf::kPanels; ++pn)
           tma_load_3d(sX + st * Cf::kXBytes + pn * Cf::kXPanel, &p.tm_x, &bar->x_full[st],
@@ -145,9 +152,9 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         long long tw = clock64();
         while (!mbar_try_wait(&bar->c_full, 0) && clock64() - tw < kWaitLimitCycles) {
         }
-        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
+        for (int j = (issued > kAsgXStages ? issued - kAsgXStages : 0); j < issued; ++j) {
           tw = clock64();
-          while (!mbar_try_wait(&bar->x_full[j & 1], (j >> 1) & 1) &&
+          while (!mbar_try_wait(&bar->x_full[j % kAsgXStages], (j / kAsgXStages) & 1) &&
                  clock64() - tw < kWaitLimitCycles) {
           }
         }
@@ -159,20 +166,20 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
       const uint32_t x_addr = smem_u32(sX), c_addr = smem_u32(sC);
       bool ok = mbar_wait(&bar->c_full, 0, abort_flag, p.status);
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(&bar->x_full[st], (j >> 1) & 1, abort_flag, p.status)) break;
-        if (!mbar_wait(&bar->s_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        const int xs = j % kAsgXStages, sb = j & 1;
+        if (!mbar_wait(&bar->x_full[xs], (j / kAsgXStages) & 1, abort_flag, p.status)) break;
+        if (!mbar_wait(&bar->s_empty[sb], ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t s_col = tmem + st * kMaxC;
+        const uint32_t s_col = tmem + sb * kMaxC;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk & 3) * 32;
-          mma_bf16_ss(s_col, sdesc_sw128(x_addr + st * Cf::kXBytes + (kk >> 2) * Cf::kXPanel + off, 16, 1024),
+          mma_bf16_ss(s_col, sdesc_sw128(x_addr + xs * Cf::kXBytes + (kk >> 2) * Cf::kXPanel + off, 16, 1024),
                       sdesc_sw128(c_addr + (kk >> 2) * Cf::kCPanel + off, 16, 1024), idesc,
                       kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bar->s_full[st]);
-        tc_commit(&bar->x_empty[st]);
+        tc_commit(&bar->s_full[sb]);
+        tc_commit(&bar->x_empty[xs]);
       }
       if (*abort_flag) {
         tc_commit(&bar->drain);
@@ -183,26 +190,31 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ argmin
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    for (int j = 0; j < n; ++j) {
-      const int st = j & 1;
+    // Four interleaved running minima per row (columns i % 4), each keeping
+    // its first minimal column; merged by (distance, column), so the result is
+    // the first column of least distance, as a single ascending scan gives.
+    const int g = warp >> 2;  // this warpgroup's tensor-memory buffer and tile parity
+    const int rl = tid & 127;
+    const uint32_t lane_base =
+        tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + static_cast<uint32_t>(g * kMaxC);
+    for (int j = g; j < n; j += 2) {
       // warp-uniform: the tensor-memory loads below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[st], (j >> 1) & 1, abort_flag, p.status)))
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[g], (j >> 1) & 1, abort_flag, p.status)))
         break;
       tc_fence_after();
-      float best = INFINITY;
-      int best_c = 0;
+      float best[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+      int best_c[4] = {0, 0, 0, 0};
       for (int ch = 0; ch < p.C / 32; ++ch) {
         uint32_t s[32];
-        tmem_ld_32x32b_x32(lane_base + st * kMaxC + ch * 32, s);
+        tmem_ld_32x32b_x32(lane_base + ch * 32, s);
         tmem_ld_wait();
         reg_fence(s);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float dist = fmaf(-2.0f, u2f(s[i]), sNorm[ch * 32 + i]);
-          if (dist < best) {  // strict: ties keep the smaller index
-            best = dist;
-            best_c = ch * 32 + i;
+          if (dist < best[i & 3]) {  // strict: ties keep the smaller column
+            best[i & 3] = dist;
+            best_c[i & 3] = ch * 32 + i;
           }
         }
       }
@@ -215,7 +227,7 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
             : "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
               "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]),
               "=r"(s[12]), "=r"(s[13]), "=r"(s[14]), "=r"(s[15])
-            : "r"(lane_base + st * kMaxC + (p.C / 32) * 32)
+            : "r"(lane_base + (p.C / 32) * 32)
             : "memory");
         tmem_ld_wait();
         reg_fence(s);
@@ -223,16 +235,24 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
         for (int i = 0; i < 16; ++i) {
           const int c = (p.C / 32) * 32 + i;
           const float dist = fmaf(-2.0f, u2f(s[i]), sNorm[c]);
-          if (dist < best) {
-            best = dist;
-            best_c = c;
+          if (dist < best[i & 3]) {
+            best[i & 3] = dist;
+            best_c[i & 3] = c;
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar->s_empty[st]);
-      const int row = (t0 + j) * 128 + tid;
-      if (row < p.N) p.assign[static_cast<size_t>(bh) * p.N + row] = best_c;
+      mbar_arrive(&bar->s_empty[g]);
+      float b = best[0];
+      int bc = best_c[0];
+#pragma unroll
+      for (int k = 1; k < 4; ++k)
+        if (best[k] < b || (best[k] == b && best_c[k] < bc)) {
+          b = best[k];
+          bc = best_c[k];
+        }
+      const int row = (t0 + j) * 128 + rl;
+      if (row < p.N) p.assign[static_cast<size_t>(bh) * p.N + row] = bc;
     }
   }
 
@@ -354,8 +374,9 @@ __global__ void sort_rank_kernel(const int32_t* __restrict__ assign, const int32
   }
 }
 
-// ------------------------------------------------------------ update
-// Members of a cluster, summed by one CTA of kSumWarps warps: warp w takes the
+// ------------------------------------------------------------ cluster sums
+// Members of a cluster, summed by one CTA of kSumWarps warps (the value
+// statistics of SVG-EAR): warp w takes the
 // w-th of kSumWarps equal runs of the cluster's sorted positions and adds its
 // rows in order (kBatch row loads in flight), lane l holding channels
 // [D/32 * l, D/32 * (l+1)); the warps' partial sums are then added in warp
@@ -411,98 +432,300 @@ __device__ __forceinline__ void sum_rows(const svg_bf16* __restrict__ x,
   }
 }
 
+// ------------------------------------------------------------ update
+// Two passes in a fixed summation order, with work per warp bounded by a
+// chunk whatever the cluster sizes. The sorted positions of a head are cut
+// into chunks of kChunkRows. Warp i of the first pass adds, in order, the rows
+// of each cluster's run inside chunk i, and stores each run's sum as the
+// partial of (chunk i, cluster c). When chunk i meets cluster c and chunk i'
+// meets cluster c' != c with i + c = i' + c', one cluster would have to end
+// past the start of the other, so slot i + c (fewer than nchunks + C slots per
+// head) is unique. The second pass adds each cluster's partials in chunk order
+// and divides by the member count.
+constexpr int kChunkRows = 256;
+constexpr int kChunkWarps = 4;
+constexpr int kChunkBatch = 16;   // rows per pipeline stage
+constexpr int kChunkStages = 4;   // stages per warp (kChunkStages - 1 batches in flight)
+
 template <int D>
-__global__ void __launch_bounds__(32 * kSumWarps)
-    kmeans_update_kernel(const svg_bf16* __restrict__ x, const int32_t* __restrict__ order,
-                         const int32_t* __restrict__ offsets, int32_t N, int32_t C,
-                         const float* __restrict__ c_in, float* __restrict__ c_out) {
+struct ChunkCfg {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kLanesPerRow = kRowBytes / 16;  // 16-byte copies per row
+  static constexpr int kRowsPerCopy = 32 / kLanesPerRow;
+  static constexpr int kStageBytes = kChunkBatch * kRowBytes;
+  static constexpr int kWarpBytes = kChunkStages * kStageBytes + kChunkRows * 4;
+  static constexpr int kSmem = kChunkWarps * kWarpBytes;
+  static_assert(kChunkBatch % kRowsPerCopy == 0, "a stage is whole copy instructions");
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One warp per chunk. The chunk's rows stream through a ring of kChunkStages
+// shared-memory stages of kChunkBatch rows (cp.async, 16 bytes per lane), so
+// the next batches are in flight while one is added; lane l adds channels
+// [D/32 * l, D/32 * (l+1)) of each row in sorted order.
+template <int D>
+__global__ void __launch_bounds__(32 * kChunkWarps)
+    kmeans_chunk_sum_kernel(const svg_bf16* __restrict__ x, const int32_t* __restrict__ order,
+                            const int32_t* __restrict__ offsets, int32_t N, int32_t C,
+                            int32_t nchunks, float* __restrict__ partial) {
+  using Cf = ChunkCfg<D>;
   constexpr int kPer = D / 32;
-  __shared__ float part[kSumWarps][D];
-  const int c = blockIdx.x, bh = blockIdx.y;
+  extern __shared__ __align__(16) uint8_t chunk_smem[];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * kChunkWarps + w;
+  const int bh = blockIdx.y;
+  if (chunk >= nchunks) return;
+  uint8_t* ring = chunk_smem + w * Cf::kWarpBytes;
+  int32_t* rows_s = reinterpret_cast<int32_t*>(ring + kChunkStages * Cf::kStageBytes);
+  const int p0 = chunk * kChunkRows, p1 = min(N, p0 + kChunkRows);
   const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
-  const int p0 = off[c], p1 = off[c + 1], cnt = p1 - p0;
-  const int q0 = p0 + static_cast<int>(static_cast<long long>(cnt) * w / kSumWarps);
-  const int q1 = p0 + static_cast<int>(static_cast<long long>(cnt) * (w + 1) / kSumWarps);
-  float acc[kPer];
+  const int32_t* ord = order + static_cast<size_t>(bh) * N;
+  for (int q = lane; q < p1 - p0; q += 32) rows_s[q] = __ldg(ord + p0 + q);
+  __syncwarp();
+  const svg_bf16* xh = x + static_cast<size_t>(bh) * N * D;
+  const int nb = (p1 - p0 + kChunkBatch - 1) / kChunkBatch;
+  const int sub = lane % Cf::kLanesPerRow, row_in_copy = lane / Cf::kLanesPerRow;
+  auto issue = [&](int bt) {
+    if (bt < nb) {
+      const uint32_t st = smem_u32(ring + (bt % kChunkStages) * Cf::kStageBytes);
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
-  sum_rows<D>(x, order, N, bh, q0, q1, lane, acc, nullptr);
+      for (int i = 0; i < kChunkBatch / Cf::kRowsPerCopy; ++i) {
+        const int u = i * Cf::kRowsPerCopy + row_in_copy;
+        const int q = bt * kChunkBatch + u;
+        if (p0 + q < p1)
+          cp_async16(st + u * Cf::kRowBytes + sub * 16,
+                     xh + static_cast<size_t>(rows_s[q]) * D + sub * 8);
+      }
+    }
+    cp_async_commit();  // an empty group past the end keeps the wait count uniform
+  };
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) part[w][lane * kPer + i] = acc[i];
-  __syncthreads();
-  if (w == 0) {
-    float* dst = c_out + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+  for (int s = 0; s < kChunkStages - 1; ++s) issue(s);
+  // the cluster of position p0: the last c with off[c] <= p0 (it is not empty)
+  int n_le = 0;
+  for (int k = lane; k <= C; k += 32) n_le += __ldg(off + k) <= p0 ? 1 : 0;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) n_le += __shfl_xor_sync(0xffffffffu, n_le, o);
+  int c = n_le - 1;
+  int next = __ldg(off + c + 1);
+  float* part = partial + static_cast<size_t>(bh) * (nchunks + C) * D + lane * kPer;
+  float sum[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) sum[i] = 0.0f;
+  for (int bt = 0; bt < nb; ++bt) {
+    issue(bt + kChunkStages - 1);  // into the stage added in the previous iteration
+    cp_async_wait<kChunkStages - 1>();
+    __syncwarp();
+    const uint8_t* st = ring + (bt % kChunkStages) * Cf::kStageBytes + lane * kPer * 2;
+#pragma unroll 4
+    for (int u = 0; u < kChunkBatch; ++u) {
+      const int p = p0 + bt * kChunkBatch + u;
+      if (p >= p1) break;
+      float v[kPer];
+      if constexpr (kPer == 4) {
+        const uint2 r = *reinterpret_cast<const uint2*>(st + u * Cf::kRowBytes);
+        v[0] = __uint_as_float(r.x << 16);
+        v[1] = __uint_as_float(r.x & 0xffff0000u);
+        v[2] = __uint_as_float(r.y << 16);
+        v[3] = __uint_as_float(r.y & 0xffff0000u);
+      } else {
+        const uint32_t r = *reinterpret_cast<const uint32_t*>(st + u * Cf::kRowBytes);
+        v[0] = __uint_as_float(r << 16);
+        v[1] = __uint_as_float(r & 0xffff0000u);
+      }
+      if (p >= next) {  // cluster c ends before p: store its run, find p's cluster
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          part[static_cast<size_t>(chunk + c) * D + i] = sum[i];
+          sum[i] = 0.0f;
+        }
+        while (p >= next && c < C - 1) next = __ldg(off + (++c) + 1);
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) sum[i] += v[i];
+    }
+    __syncwarp();  // every lane is done with this stage before it is refilled
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) part[static_cast<size_t>(chunk + c) * D + i] = sum[i];
+}
+
+template <int D>
+__global__ void __launch_bounds__(32 * kChunkWarps)
+    kmeans_mean_kernel(const float* __restrict__ partial, const int32_t* __restrict__ offsets,
+                       int32_t C, int32_t nchunks, const float* __restrict__ c_in,
+                       float* __restrict__ c_out) {
+  constexpr int kPer = D / 32;
+  constexpr int kInFlight = 8;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x * kChunkWarps + (threadIdx.x >> 5);
+  const int bh = blockIdx.y;
+  if (c >= C) return;
+  const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
+  const int p0 = __ldg(off + c), p1 = __ldg(off + c + 1);
+  float* dst = c_out + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
+  if (p1 <= p0) {
     const float* prev = c_in + (static_cast<size_t>(bh) * C + c) * D + lane * kPer;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      float tot = 0.0f;
+    for (int i = 0; i < kPer; ++i) dst[i] = prev[i];
+    return;
+  }
+  const int i0 = p0 / kChunkRows, i1 = (p1 - 1) / kChunkRows;
+  const float* part = partial + static_cast<size_t>(bh) * (nchunks + C) * D + lane * kPer;
+  float tot[kPer];
 #pragma unroll
-      for (int ww = 0; ww < kSumWarps; ++ww) tot += part[ww][lane * kPer + i];
-      dst[i] = cnt > 0 ? __fdiv_rn(tot, static_cast<float>(cnt)) : prev[i];
+  for (int i = 0; i < kPer; ++i) tot[i] = 0.0f;
+  for (int ib = i0; ib <= i1; ib += kInFlight) {
+    float v[kInFlight][kPer];
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u)
+      if (ib + u <= i1) {
+        const float* src = part + static_cast<size_t>(ib + u + c) * D;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) v[u][i] = src[i];
+      }
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u) {
+      if (ib + u > i1) break;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) tot[i] += v[u][i];
     }
   }
+  const float n = static_cast<float>(p1 - p0);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) dst[i] = __fdiv_rn(tot[i], n);
 }
 
 // ------------------------------------------------------------ selection
-// One CTA per (bh, query cluster a); thread b per key cluster.
+// One CTA per (bh, group of kSelGroup query clusters); the group's centroids
+// are staged in shared memory. Each warp forms the kSelGroup dot products of
+// its share of the key clusters, lane l taking channels l, l + 32, ... (the
+// key centroid is read once per group, coalesced) and the lanes' partial sums
+// added by a butterfly. Thread b then handles key cluster b: for each query
+// cluster of the group the weights, their maximum and their sum are formed as
+// for a lone cluster.
 // With disp != nullptr (SVG-EAR), a skipped cluster is kept anyway when its
 // error estimate w_b * disp_b exceeds tau.
+constexpr int kSelGroup = 8;
+
 __global__ void select_kernel(const float* __restrict__ cq, const float* __restrict__ ck,
                               const int32_t* __restrict__ offsets_k, int32_t D, int32_t Cq,
                               int32_t Ck, float scale, float top_p, const float* __restrict__ disp,
                               float tau, uint32_t* __restrict__ sel) {
-  extern __shared__ float w[];  // [Ck] weights, then [32] reduction slots
-  float* red = w + Ck;
-  const int a = blockIdx.x, bh = blockIdx.y;
+  // [kSelGroup][Ck] weights (first the dot products), [kSelGroup][32]
+  // reduction slots, then [kSelGroup][D] query centroids
+  extern __shared__ float w[];
+  float* red = w + kSelGroup * Ck;
+  float* xs = red + kSelGroup * 32;
+  const int a0 = blockIdx.x * kSelGroup, bh = blockIdx.y;
+  const int na = min(kSelGroup, Cq - a0);
   const int b = threadIdx.x;
   const int lane = b & 31, wid = b >> 5, nw = blockDim.x >> 5;
   const int words = (Ck + 31) / 32;
-  float z = -INFINITY;
+  const int32_t* off = offsets_k + static_cast<size_t>(bh) * (Ck + 1);
+  {
+    const float* x = cq + (static_cast<size_t>(bh) * Cq + a0) * D;
+    for (int i = b; i < kSelGroup * D; i += blockDim.x) xs[i] = i < na * D ? x[i] : 0.0f;
+  }
+  __syncthreads();
+  for (int kb = wid; kb < Ck; kb += nw) {
+    if (off[kb + 1] - off[kb] <= 0) continue;  // warp-uniform
+    const float* y = ck + (static_cast<size_t>(bh) * Ck + kb) * D;
+    float acc[kSelGroup];
+#pragma unroll
+    for (int g = 0; g < kSelGroup; ++g) acc[g] = 0.0f;
+    for (int i = lane; i < D; i += 32) {
+      const float yi = y[i];
+#pragma unroll
+      for (int g = 0; g < kSelGroup; ++g) acc[g] = fmaf(xs[g * D + i], yi, acc[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < kSelGroup; ++g) {
+      for (int o = 16; o > 0; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int g = 0; g < kSelGroup; ++g) w[g * Ck + kb] = acc[g];
+    }
+  }
+  __syncthreads();
+  float z[kSelGroup];
+#pragma unroll
+  for (int g = 0; g < kSelGroup; ++g) z[g] = -INFINITY;
   int size = 0;
   if (b < Ck) {
-    const int32_t* off = offsets_k + static_cast<size_t>(bh) * (Ck + 1);
     size = off[b + 1] - off[b];
     if (size > 0) {
-      const float* x = cq + (static_cast<size_t>(bh) * Cq + a) * D;
-      const float* y = ck + (static_cast<size_t>(bh) * Ck + b) * D;
-      float dot = 0.0f;
-      for (int i = 0; i < D; ++i) dot = fmaf(x[i], y[i], dot);
-      z = fmaf(scale, dot, logf(static_cast<float>(size)));
+      const float ls = logf(static_cast<float>(size));
+#pragma unroll
+      for (int g = 0; g < kSelGroup; ++g) z[g] = fmaf(scale, w[g * Ck + b], ls);
     }
   }
-  // block max
-  float m = z;
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[wid] = m;
-  __syncthreads();
-  m = -INFINITY;
-  for (int i = 0; i < nw; ++i) m = fmaxf(m, red[i]);
-  __syncthreads();
-  const float e = (b < Ck && size > 0) ? expf(z - m) : 0.0f;
-  // block sum in a fixed order
-  float s = e;
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) red[wid] = s;
-  __syncthreads();
-  float tot = 0.0f;
-  for (int i = 0; i < nw; ++i) tot += red[i];
-  const float wb = e / tot;
-  if (b < Ck) w[b] = wb;
-  __syncthreads();
-  bool keep = false;
-  if (b < Ck && size > 0) {
-    // weight of the clusters ranked before b (descending weight, ties by index)
-    float before = 0.0f;
-    for (int i = 0; i < Ck; ++i) {
-      const float wi = w[i];
-      if (wi > wb || (wi == wb && i < b)) before += wi;
-    }
-    keep = before < top_p;
-    if (!keep && disp != nullptr) keep = wb * disp[static_cast<size_t>(bh) * Ck + b] > tau;
+  __syncthreads();  // the dot products are read; w now takes the weights
+  // block maxima
+  float m[kSelGroup];
+#pragma unroll
+  for (int g = 0; g < kSelGroup; ++g) {
+    m[g] = z[g];
+    for (int o = 16; o > 0; o >>= 1) m[g] = fmaxf(m[g], __shfl_xor_sync(0xffffffffu, m[g], o));
+    if (lane == 0) red[g * 32 + wid] = m[g];
   }
-  const unsigned bits = __ballot_sync(0xffffffffu, keep);
-  if (lane == 0 && wid < words) sel[(static_cast<size_t>(bh) * Cq + a) * words + wid] = bits;
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < kSelGroup; ++g) {
+    m[g] = -INFINITY;
+    for (int i = 0; i < nw; ++i) m[g] = fmaxf(m[g], red[g * 32 + i]);
+  }
+  __syncthreads();
+  // block sums in a fixed order
+  float e[kSelGroup];
+#pragma unroll
+  for (int g = 0; g < kSelGroup; ++g) {
+    e[g] = (b < Ck && size > 0) ? expf(z[g] - m[g]) : 0.0f;
+    float s = e[g];
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[g * 32 + wid] = s;
+  }
+  __syncthreads();
+  float wb[kSelGroup];
+#pragma unroll
+  for (int g = 0; g < kSelGroup; ++g) {
+    float tot = 0.0f;
+    for (int i = 0; i < nw; ++i) tot += red[g * 32 + i];
+    wb[g] = e[g] / tot;
+    if (b < Ck) w[g * Ck + b] = wb[g];
+  }
+  __syncthreads();
+  const float db = (disp != nullptr && b < Ck) ? disp[static_cast<size_t>(bh) * Ck + b] : 0.0f;
+#pragma unroll
+  for (int g = 0; g < kSelGroup; ++g) {
+    if (g >= na) break;
+    bool keep = false;
+    if (b < Ck && size > 0) {
+      // weight of the clusters ranked before b (descending weight, ties by index)
+      const float* wg = w + g * Ck;
+      float before = 0.0f;
+      for (int i = 0; i < Ck; ++i) {
+        const float wi = wg[i];
+        if (wi > wb[g] || (wi == wb[g] && i < b)) before += wi;
+      }
+      keep = before < top_p;
+      if (!keep && disp != nullptr) keep = wb[g] * db > tau;
+    }
+    const unsigned bits = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0 && wid < words) sel[(static_cast<size_t>(bh) * Cq + a0 + g) * words + wid] = bits;
+  }
 }
 
 // ------------------------------------------------------------ tile CSR
@@ -1021,6 +1244,7 @@ size_t kmeans_workspace_bytes(int32_t BH, int32_t N, int32_t D, int32_t C) {
   add(static_cast<size_t>(BH) * C * 4);            // norms
   add(static_cast<size_t>(BH) * nblk * C * 4);     // sort histograms
   add(static_cast<size_t>(BH) * C * D * 4);        // the other centroid buffer
+  add(static_cast<size_t>(BH) * ((N + kChunkRows - 1) / kChunkRows + C) * D * 4);  // run sums
   return (b + 255) / 256 * 256;
 }
 
@@ -1030,6 +1254,7 @@ struct KWs {
   float* norms;
   int32_t* hist;
   float* cent2;
+  float* partial;
 };
 KWs carve(void* ws, int32_t BH, int32_t N, int32_t D, int32_t C) {
   const size_t nblk = (static_cast<size_t>(N) + kSortRows - 1) / kSortRows;
@@ -1046,6 +1271,8 @@ KWs carve(void* ws, int32_t BH, int32_t N, int32_t D, int32_t C) {
   w.norms = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * C * 4));
   w.hist = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nblk * C * 4));
   w.cent2 = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * C * D * 4));
+  w.partial = reinterpret_cast<float*>(
+      take(static_cast<size_t>(BH) * ((N + kChunkRows - 1) / kChunkRows + C) * D * 4));
   return w;
 }
 
@@ -1105,14 +1332,31 @@ cudaError_t launch_cluster_sort(int32_t BH, int32_t N, int32_t C, const int32_t*
 
 cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
                                  const int32_t* order, const int32_t* offsets, const float* c_in,
-                                 float* c_out, cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>(C), static_cast<unsigned>(BH));
-  if (D == 128)
-    kmeans_update_kernel<128><<<grid, 32 * kSumWarps, 0, stream>>>(x, order, offsets, N, C, c_in,
-                                                                   c_out);
-  else
-    kmeans_update_kernel<64><<<grid, 32 * kSumWarps, 0, stream>>>(x, order, offsets, N, C, c_in,
-                                                                  c_out);
+                                 float* c_out, void* ws, cudaStream_t stream) {
+  const KWs w = carve(ws, BH, N, D, C);
+  const int nchunks = (N + kChunkRows - 1) / kChunkRows;
+  const dim3 g_sum(static_cast<unsigned>((nchunks + kChunkWarps - 1) / kChunkWarps),
+                   static_cast<unsigned>(BH));
+  const dim3 g_mean(static_cast<unsigned>((C + kChunkWarps - 1) / kChunkWarps),
+                    static_cast<unsigned>(BH));
+  cudaError_t e;
+  if (D == 128) {
+    e = cudaFuncSetAttribute(kmeans_chunk_sum_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ChunkCfg<128>::kSmem);
+    if (e != cudaSuccess) return e;
+    kmeans_chunk_sum_kernel<128><<<g_sum, 32 * kChunkWarps, ChunkCfg<128>::kSmem, stream>>>(
+        x, order, offsets, N, C, nchunks, w.partial);
+    kmeans_mean_kernel<128><<<g_mean, 32 * kChunkWarps, 0, stream>>>(w.partial, offsets, C,
+                                                                     nchunks, c_in, c_out);
+  } else {
+    e = cudaFuncSetAttribute(kmeans_chunk_sum_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ChunkCfg<64>::kSmem);
+    if (e != cudaSuccess) return e;
+    kmeans_chunk_sum_kernel<64><<<g_sum, 32 * kChunkWarps, ChunkCfg<64>::kSmem, stream>>>(
+        x, order, offsets, N, C, nchunks, w.partial);
+    kmeans_mean_kernel<64><<<g_mean, 32 * kChunkWarps, 0, stream>>>(w.partial, offsets, C, nchunks,
+                                                                    c_in, c_out);
+  }
   return cudaGetLastError();
 }
 
@@ -1140,7 +1384,7 @@ cudaError_t launch_kmeans(int32_t BH, int32_t N, int32_t D, int32_t C, int32_t i
     if ((e = launch_cluster_sort(BH, N, C, assign, order, offsets, ws, D, status, stream)) !=
         cudaSuccess)
       return e;
-    if ((e = launch_kmeans_update(BH, N, D, C, x, order, offsets, bufs[cur], bufs[cur ^ 1],
+    if ((e = launch_kmeans_update(BH, N, D, C, x, order, offsets, bufs[cur], bufs[cur ^ 1], ws,
                                   stream)) != cudaSuccess)
       return e;
     cur ^= 1;
@@ -1159,9 +1403,14 @@ cudaError_t launch_select_clusters(int32_t BH, int32_t D, int32_t Cq, int32_t Ck
                                    const int32_t* offsets_k, const float* disp, float tau,
                                    uint32_t* sel, cudaStream_t stream) {
   const int threads = (Ck + 31) / 32 * 32;
-  const size_t sm = (static_cast<size_t>(Ck) + 32) * sizeof(float);
-  select_kernel<<<dim3(Cq, BH), threads, sm, stream>>>(cq, ck, offsets_k, D, Cq, Ck, scale, top_p,
-                                                      disp, tau, sel);
+  const size_t sm = static_cast<size_t>(kSelGroup) * (Ck + 32 + D) * sizeof(float);
+  if (sm > 227 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sm));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>((Cq + kSelGroup - 1) / kSelGroup), static_cast<unsigned>(BH));
+  select_kernel<<<grid, threads, sm, stream>>>(cq, ck, offsets_k, D, Cq, Ck, scale, top_p, disp,
+                                               tau, sel);
   return cudaGetLastError();
 }
 
