@@ -318,34 +318,57 @@ __global__ void sort_hist_kernel(const int32_t* __restrict__ assign, int32_t N, 
 
 // Per head: offsets[c] = rows in clusters < c; hist becomes each block's first
 // sorted position per cluster (offsets[c] + rows of earlier blocks in c).
-__global__ void sort_scan_kernel(int32_t* __restrict__ hist, int32_t N, int32_t C, int32_t nblk,
-                                 int32_t* __restrict__ offsets) {
-  extern __shared__ int tot[];
+// Thread c walks cluster c's column of the histogram, kScanBatch blocks of
+// loads in flight; the cluster totals are scanned across the CTA (C <= 256 =
+// blockDim.x).
+constexpr int kScanBatch = 16;
+
+__global__ void __launch_bounds__(256)
+    sort_scan_kernel(int32_t* __restrict__ hist, int32_t N, int32_t C, int32_t nblk,
+                     int32_t* __restrict__ offsets) {
+  __shared__ int warp_tot[8];
   const int bh = blockIdx.x;
+  const int c = threadIdx.x, lane = c & 31, wid = c >> 5;
   int32_t* h = hist + static_cast<size_t>(bh) * nblk * C;
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int v = h[static_cast<size_t>(b) * C + c];
-      h[static_cast<size_t>(b) * C + c] = run;
-      run += v;
+  int run = 0;
+  if (c < C) {
+    for (int b0 = 0; b0 < nblk; b0 += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        v[i] = b0 + i < nblk ? h[static_cast<size_t>(b0 + i) * C + c] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) {
+        if (b0 + i < nblk) h[static_cast<size_t>(b0 + i) * C + c] = run;
+        run += v[i];
+      }
     }
-    tot[c] = run;
   }
+  // exclusive scan of the cluster totals over c
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int c = 0; c < C; ++c) {
-      const int v = tot[c];
-      tot[c] = run;
-      offsets[static_cast<size_t>(bh) * (C + 1) + c] = run;
-      run += v;
+  int before = 0;
+  for (int w = 0; w < wid; ++w) before += warp_tot[w];
+  const int first = before + incl - run;  // rows in clusters < c
+  if (c < C) offsets[static_cast<size_t>(bh) * (C + 1) + c] = first;
+  if (c == C - 1) offsets[static_cast<size_t>(bh) * (C + 1) + C] = first + run;
+  if (c < C) {
+    for (int b0 = 0; b0 < nblk; b0 += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        v[i] = b0 + i < nblk ? h[static_cast<size_t>(b0 + i) * C + c] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        if (b0 + i < nblk) h[static_cast<size_t>(b0 + i) * C + c] = v[i] + first;
     }
-    offsets[static_cast<size_t>(bh) * (C + 1) + C] = run;
   }
-  __syncthreads();
-  for (int c = threadIdx.x; c < C; c += blockDim.x)
-    for (int b = 0; b < nblk; ++b) h[static_cast<size_t>(b) * C + c] += tot[c];
 }
 
 // One warp per block: walks its rows in order, 32 at a time, and gives each
@@ -1324,7 +1347,7 @@ cudaError_t launch_cluster_sort(int32_t BH, int32_t N, int32_t C, const int32_t*
   sort_hist_kernel<<<dim3(nblk, BH), 256, sm, stream>>>(assign, N, C, nblk, w.hist, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  sort_scan_kernel<<<BH, 256, sm, stream>>>(w.hist, N, C, nblk, offsets);
+  sort_scan_kernel<<<BH, 256, 0, stream>>>(w.hist, N, C, nblk, offsets);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   sort_rank_kernel<<<dim3(nblk, BH), 32, sm, stream>>>(assign, w.hist, N, C, nblk, order);
   return cudaGetLastError();
