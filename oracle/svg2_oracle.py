@@ -186,16 +186,17 @@ def selection_weights(cq, ck, sizes_k, scale) -> np.ndarray:
 # block mask and attention on the sorted layouts
 # ---------------------------------------------------------------------------
 def semantic_block_mask(offsets_q: np.ndarray, offsets_k: np.ndarray, sel: np.ndarray,
-                        block_q: int, block_k: int) -> np.ndarray:
+                        block_q: int, block_k: int, tiles=None) -> np.ndarray:
     """bool [nQB, nKB]: tile pair (r, c) is on iff some sorted query position of
     tile r and sorted key position of tile c have sel[cluster(q), cluster(k)],
-    evaluated token pair by token pair (brute force over positions)."""
+    evaluated token pair by token pair (brute force over positions). With
+    `tiles`, only those query tiles are evaluated (the other rows stay off)."""
     cq = cluster_of_position(offsets_q)
     ck = cluster_of_position(offsets_k)
     Nq, Nk = cq.size, ck.size
     nqb, nkb = n_blocks(Nq, block_q), n_blocks(Nk, block_k)
     bm = np.zeros((nqb, nkb), dtype=bool)
-    for r in range(nqb):
+    for r in (range(nqb) if tiles is None else sorted(set(int(t) for t in tiles))):
         rows = cq[r * block_q:min(Nq, (r + 1) * block_q)]
         allowed = sel[rows][:, ck]  # [rows of the tile, Nk]
         any_key = allowed.any(axis=0)

@@ -361,3 +361,103 @@ def test_semantic_layer_end_to_end_on_planted_frames(svg):
         assert_close(got[0, h], want, f"semantic layer head {h}")
         print(f"SEMANTIC head {h}: tile density {bm.mean():.4f}")
     status_clean()
+
+
+def _unpack_sel(sel, Ck):
+    bits = sel.cpu().numpy().view(np.uint32)
+    return (((bits[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1)
+            .reshape(bits.shape[0], bits.shape[1], -1)[..., :Ck].astype(bool))
+
+
+@pytest.mark.parametrize("ear_tau", [None, 0.01], ids=["svg2", "ear"])
+def test_semantic_layer_full_size_sampled_rows(svg, ear_tau):
+    """HunyuanVideo-shaped length (N = 119 056, d = 128), 2 heads of the seeded
+    layer, C = 256 clusters, 10 iterations, top-p 0.9, with and without SVG-EAR
+    routing: every part of the plan the GPU builds is checked against what
+    defines it, and the output against the oracle's attention over that plan
+    on sampled rows.
+      - order and offsets: the stable cluster order of the GPU's own assignment;
+      - selection: each query cluster's kept set is a valid top-p prefix of the
+        oracle's weights from the GPU's centroids (with routing: every cluster
+        whose estimate clears tau is kept, and what is kept otherwise is a valid
+        prefix);
+      - value statistics (SVG-EAR): the oracle's means and dispersions;
+      - tile CSR: bit-exact against the oracle's block mask of that plan on
+        sampled query tiles (the first, the ragged last, random ones);
+      - output: element-wise within the attention bars on sampled rows."""
+    import svg_inputs as SI
+    from video_dit_spatial_b200.layer import SemanticSparseLayer
+    wl = SI.HUNYUAN.replace(H=2, n_spatial=1)
+    q, k, v = SI.make_qkv(wl)
+    B, H, N, d, C, top_p = 1, 2, wl.N, wl.d, 256, 0.9
+    layer = SemanticSparseLayer(B, H, N, d, Cq=C, Ck=C, iters=10, top_p=top_p, ear_tau=ear_tau)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device="cuda")
+    layer.forward(q.cuda(), k.cuda(), v.cuda(), o)
+    torch.cuda.synchronize()
+    scale = layer.scale
+    got = to_f64(o)
+    sel_all = _unpack_sel(layer.sel, C)
+    rp, ci, nqb = layer.row_ptr.cpu().numpy(), layer.col_idx.cpu().numpy(), layer.nqb
+    rng = np.random.default_rng(77 if ear_tau is None else 78)
+    for h in range(H):
+        qn, kn, vn = to_f64(q[0, h]), to_f64(k[0, h]), to_f64(v[0, h])
+        plan = {}
+        for name in ("q", "k"):
+            a = getattr(layer, "assign_" + name)[h].cpu().numpy()
+            order = getattr(layer, "order_" + name)[h].cpu().numpy()
+            offs = getattr(layer, "offsets_" + name)[h].cpu().numpy()
+            want_order, want_offs = S2.cluster_permutation(a, C)
+            assert np.array_equal(order, want_order) and np.array_equal(offs, want_offs), name
+            plan[name] = (order, offs)
+        (oq_, offq), (ok_, offk) = plan["q"], plan["k"]
+        cq = layer.cq[h].cpu().numpy().astype(np.float64)
+        ck = layer.ck[h].cpu().numpy().astype(np.float64)
+        sizes = np.diff(offk)
+        w = S2.selection_weights(cq, ck, sizes, scale)
+        sel = sel_all[h]
+        if ear_tau is None:
+            for a in range(C):
+                if offq[a + 1] > offq[a]:
+                    assert _selection_valid(w[a], sizes, sel[a], top_p), f"head {h} cluster {a}"
+        else:
+            vbar = layer.vbar[h].cpu().numpy().astype(np.float64)
+            disp = layer.disp[h].cpu().numpy().astype(np.float64)
+            want_vbar, want_disp = S2.cluster_value_stats(vn, ok_, offk)
+            np.testing.assert_allclose(vbar, want_vbar, rtol=1e-4, atol=1e-5)
+            np.testing.assert_allclose(disp, want_disp, rtol=1e-4, atol=1e-5)
+            est = w * disp[None, :]
+            must = (est > ear_tau * (1 + 1e-4)) & (sizes > 0)[None, :]
+            may = est > ear_tau * (1 - 1e-4)
+            routed_only = 0
+            for a in range(C):
+                if offq[a + 1] <= offq[a]:
+                    continue
+                assert not np.any(must[a] & ~sel[a]), f"head {h} cluster {a}: a routed pair is missing"
+                # what is kept beyond the routable clusters is a top-p prefix
+                base = sel[a] & ~may[a]
+                live = sizes > 0
+                out = live & ~sel[a]
+                if np.any(base):
+                    assert w[a][base].min() >= (w[a][out].max() if np.any(out) else -1) - 1e-5
+                    assert w[a][base].sum() - w[a][base].min() < top_p + 1e-5
+                assert w[a][sel[a] & live].sum() >= top_p - 1e-5
+                routed_only += int(np.sum(sel[a] & may[a] & ~must[a]))
+        # tile CSR on sampled query tiles, and the output on sampled rows
+        pos = np.unique(np.concatenate([np.arange(4), np.arange(N - 4, N),
+                                        rng.choice(N, 40, replace=False)]))
+        tiles = np.unique(np.concatenate([pos // 128, rng.choice(nqb, 12, replace=False)]))
+        bm = S2.semantic_block_mask(offq, offk, sel, 128, 128, tiles=tiles)
+        for r in tiles:
+            row = h * nqb + r
+            assert np.array_equal(ci[rp[row]:rp[row + 1]], np.nonzero(bm[r])[0]), (h, r)
+        rows = oq_[pos]
+        if ear_tau is None:
+            want, _ = S2.semantic_attention_rows(qn, kn, vn, oq_, ok_, bm, 128, 128, scale, rows)
+        else:
+            want = S2.ear_attention_rows(qn, kn, vn, oq_, ok_, offk, ck, vbar, bm, 128, 128,
+                                         scale, rows)
+        density = float(np.diff(rp[h * nqb:(h + 1) * nqb + 1]).sum()) / (nqb * layer.nkb)
+        print(f"SVG2-FULL {'ear' if ear_tau else 'svg2'} head {h}: tile density {density:.3f}, "
+              f"{len(tiles)} tiles and {len(rows)} rows checked")
+        assert_close(got[0, h][rows], want, f"SVG2 full size {'ear' if ear_tau else 'svg2'} head {h}")
+    status_clean()
