@@ -559,7 +559,7 @@ svg_status svg2_kmeans_step(int32_t BH, int32_t N, int32_t d, int32_t C, const s
       svg::launch_cluster_sort(BH, N, C, assign, order, offsets, workspace, d, status, s) !=
           cudaSuccess ||
       svg::launch_kmeans_update(BH, N, d, C, x, order, offsets, centroids_in, centroids_out,
-                                workspace, s) !=
+                                workspace, status, s) !=
           cudaSuccess)
     return SVG_ERR_CUDA;
   return SVG_OK;

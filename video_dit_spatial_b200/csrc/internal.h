@@ -161,7 +161,7 @@ cudaError_t launch_cluster_sort(int32_t BH, int32_t N, int32_t C, const int32_t*
                                 cudaStream_t stream);
 cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
                                  const int32_t* order, const int32_t* offsets, const float* c_in,
-                                 float* c_out, void* ws, cudaStream_t stream);
+                                 float* c_out, void* ws, int* status, cudaStream_t stream);
 cudaError_t launch_select_clusters(int32_t BH, int32_t D, int32_t Cq, int32_t Ck, float scale,
                                    float top_p, const float* cq, const float* ck,
                                    const int32_t* offsets_k, const float* disp, float tau,

@@ -500,7 +500,7 @@ template <int D>
 __global__ void __launch_bounds__(32 * kChunkWarps)
     kmeans_chunk_sum_kernel(const svg_bf16* __restrict__ x, const int32_t* __restrict__ order,
                             const int32_t* __restrict__ offsets, int32_t N, int32_t C,
-                            int32_t nchunks, float* __restrict__ partial) {
+                            int32_t nchunks, float* __restrict__ partial, int* status) {
   using Cf = ChunkCfg<D>;
   constexpr int kPer = D / 32;
   extern __shared__ __align__(16) uint8_t chunk_smem[];
@@ -513,7 +513,14 @@ __global__ void __launch_bounds__(32 * kChunkWarps)
   const int p0 = chunk * kChunkRows, p1 = min(N, p0 + kChunkRows);
   const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
   const int32_t* ord = order + static_cast<size_t>(bh) * N;
-  for (int q = lane; q < p1 - p0; q += 32) rows_s[q] = __ldg(ord + p0 + q);
+  for (int q = lane; q < p1 - p0; q += 32) {
+    int r = __ldg(ord + p0 + q);
+    if (r < 0 || r >= N) {  // only if an earlier step failed: flag it, read row 0
+      atomicOr(status, kDevErrBounds);
+      r = 0;
+    }
+    rows_s[q] = r;
+  }
   __syncwarp();
   const svg_bf16* xh = x + static_cast<size_t>(bh) * N * D;
   const int nb = (p1 - p0 + kChunkBatch - 1) / kChunkBatch;
@@ -539,7 +546,9 @@ __global__ void __launch_bounds__(32 * kChunkWarps)
   for (int k = lane; k <= C; k += 32) n_le += __ldg(off + k) <= p0 ? 1 : 0;
 #pragma unroll
   for (int o = 16; o; o >>= 1) n_le += __shfl_xor_sync(0xffffffffu, n_le, o);
-  int c = n_le - 1;
+  // (C - 1 at most: the positions of rows an earlier failed step left unsorted
+  // lie past off[C])
+  int c = min(n_le - 1, C - 1);
   int next = __ldg(off + c + 1);
   float* part = partial + static_cast<size_t>(bh) * (nchunks + C) * D + lane * kPer;
   float sum[kPer];
@@ -976,18 +985,24 @@ __global__ void to_bf16_kernel(const float* __restrict__ x, int64_t n, svg_bf16*
     y[i] = static_cast<svg_bf16>(pack_bf16x2(x[i], 0.0f) & 0xffffu);
 }
 
-// Centroid compensation of one sorted query tile (128 rows) of head bh:
+// Centroid compensation of sorted query tiles (128 rows) of head bh:
 //   bias_b = log2(n_b), n_b = keys of cluster b outside the tile's computed key
 //            tiles (-inf when none);
 //   S = Q kbar^T (tcgen05, 128 x Ck), z_b = S_b * scale * log2(e) + bias_b,
 //   P = 2^(z - max z) (bf16, in tensor memory), O_c = P vbar (tcgen05);
 // then merged with the block-sparse output of the same rows through its
 // log-sum-exp: O = (O_s e^lse + O_c 2^m) / (e^lse + sum P 2^m), in place.
+// Persistent: CTA i takes the consecutive tiles [T0, T1) of the (bh, tile)
+// order, loads a head's bf16 centroids and value means once, and streams the
+// query tiles through two shared-memory buffers. Per tile each of s_full,
+// p_full, o_full and o_empty completes once (kv_free once per change of head,
+// c_full once per load), and every wait is on a phase that the waiter's own
+// earlier step must precede, so no barrier runs two phases ahead of a waiter.
 constexpr int kEarThreads = 192;  // warps 0-3 softmax / merge, 4 producer, 5 MMA
 constexpr int kEarMaxTiles = 4096;
 
 struct EarBarriers {
-  uint64_t c_full, q_full, s_full, p_full, o_full, drain;
+  uint64_t c_full, kv_free, q_full[2], q_empty[2], s_full, p_full, o_full, o_empty, drain;
   uint32_t tmem_base;
   int abort_flag;
   uint32_t tiles[kEarMaxTiles / 32];
@@ -1002,9 +1017,9 @@ struct EarCfg {
   static constexpr int kQBytes = kPanels * kQPanel;
   static constexpr int kOffK = 0;               // kbar (K-major operand of S)
   static constexpr int kOffV = kOffK + kCBytes;  // vbar (MN-major operand of O)
-  static constexpr int kOffQ = kOffV + kCBytes;
-  static constexpr int kOffBias = kOffQ + kQBytes;
-  static constexpr int kOffBar = kOffBias + kMaxC * 4;
+  static constexpr int kOffQ = kOffV + kCBytes;  // two query tiles
+  static constexpr int kOffBias = kOffQ + 2 * kQBytes;  // two tiles' biases
+  static constexpr int kOffBar = kOffBias + 2 * kMaxC * 4;
   static constexpr int kBarBytes = (static_cast<int>(sizeof(EarBarriers)) + 127) / 128 * 128;
   static constexpr int kUsed = kOffBar + kBarBytes + 1024;
   static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
@@ -1022,9 +1037,39 @@ struct __align__(64) EarParams {
   svg_bf16* os;              // [BH, N, D] sorted sparse output, overwritten
   const float* lse;          // [BH, N] natural log
   int* status;
-  int32_t N, C, bk, nqb, nkb;
+  int32_t BH, N, C, bk, nqb, nkb;
   float scale_log2;
 };
+
+// 16 columns of 32-bit tensor memory of this warp's 32 lanes
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Barrier `id` over `count` threads that also returns the OR of `pred` over them.
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 template <int D>
 __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __grid_constant__ EarParams p) {
@@ -1039,7 +1084,10 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
   EarBarriers* bar = reinterpret_cast<EarBarriers*>(smem + Cf::kOffBar);
   volatile int* abort_flag = &bar->abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int r = blockIdx.x, bh = blockIdx.y;
+  // this CTA's tiles: [T0, T0 + n) of the order u = bh * nqb + r
+  const long long total = static_cast<long long>(p.BH) * p.nqb;
+  const int T0 = static_cast<int>(total * blockIdx.x / gridDim.x);
+  const int n = static_cast<int>(total * (blockIdx.x + 1) / gridDim.x) - T0;
 
   if (warp == 0) {
     tmem_alloc(&bar->tmem_base, 512);
@@ -1048,88 +1096,109 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
   }
   if (tid == 32) {
     mbar_init(&bar->c_full, 1);
-    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->kv_free, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar->q_full[b], 1);
+      mbar_init(&bar->q_empty[b], 1);
+    }
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->p_full, 128);
     mbar_init(&bar->o_full, 1);
+    mbar_init(&bar->o_empty, 128);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_mbar_init();
-  }
-  // the tile's computed key tiles as a bitmap
-  const int tw = (p.nkb + 31) / 32;
-  for (int i = tid; i < tw; i += kEarThreads) bar->tiles[i] = 0u;
-  __syncthreads();
-  const int row = bh * p.nqb + r;
-  const int c0 = p.row_ptr[row], c1 = p.row_ptr[row + 1];
-  for (int i = c0 + tid; i < c1; i += kEarThreads) {
-    const int t = p.col_idx[i];
-    if (t >= 0 && t < p.nkb) atomicOr(&bar->tiles[t >> 5], 1u << (t & 31));
-    else atomicOr(p.status, kDevErrBounds);
-  }
-  __syncthreads();
-  // bias_b = log2 of the cluster's uncovered keys
-  const int32_t* off = p.offsets_k + static_cast<size_t>(bh) * (p.C + 1);
-  for (int b = tid; b < p.C; b += kEarThreads) {
-    const int k0 = off[b], k1 = off[b + 1];
-    int covered = 0;
-    if (k1 > k0) {
-      for (int t = k0 / p.bk; t <= (k1 - 1) / p.bk; ++t) {
-        if ((bar->tiles[t >> 5] >> (t & 31)) & 1u) {
-          const int lo = max(k0, t * p.bk), hi = min(k1, (t + 1) * p.bk);
-          covered += hi - lo;
-        }
-      }
-    }
-    const int n = k1 - k0 - covered;
-    sBias[b] = n > 0 ? __log2f(static_cast<float>(n)) : -INFINITY;
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
   if (warp == 4) {
+    // ------------------------------------------------------------ producer
     if (lane_id() == 0) {
-      mbar_arrive_expect_tx(&bar->c_full, static_cast<uint32_t>(2 * p.C * D * 2));
-      for (int pn = 0; pn < Cf::kPanels; ++pn) {
-        tma_load_3d(sK + pn * Cf::kCPanel, &p.tm_kb, &bar->c_full, pn * 64, 0, bh);
-        tma_load_3d(sV + pn * Cf::kCPanel, &p.tm_vb, &bar->c_full, pn * 64, 0, bh);
+      int cur = -1, loads = 0, q_issued = 0;
+      bool ok = true;
+      for (int it = 0; it < n; ++it) {
+        const int u = T0 + it, bh = u / p.nqb, r = u - bh * p.nqb;
+        if (bh != cur) {
+          // the previous head's last product has read its centroids
+          if (loads > 0 && !mbar_wait(&bar->kv_free, (loads - 1) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar->c_full, static_cast<uint32_t>(2 * p.C * D * 2));
+          for (int pn = 0; pn < Cf::kPanels; ++pn) {
+            tma_load_3d(sK + pn * Cf::kCPanel, &p.tm_kb, &bar->c_full, pn * 64, 0, bh);
+            tma_load_3d(sV + pn * Cf::kCPanel, &p.tm_vb, &bar->c_full, pn * 64, 0, bh);
+          }
+          ++loads;
+          cur = bh;
+        }
+        const int b = it & 1;
+        if (!mbar_wait(&bar->q_empty[b], ((it >> 1) & 1) ^ 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bar->q_full[b], Cf::kQBytes);
+        for (int pn = 0; pn < Cf::kPanels; ++pn)
+          tma_load_3d(sQ + b * Cf::kQBytes + pn * Cf::kQPanel, &p.tm_q, &bar->q_full[b],
+                      pn * 64, r * 128, bh);
+        q_issued = it + 1;
       }
-      mbar_arrive_expect_tx(&bar->q_full, Cf::kQBytes);
-      for (int pn = 0; pn < Cf::kPanels; ++pn)
-        tma_load_3d(sQ + pn * Cf::kQPanel, &p.tm_q, &bar->q_full, pn * 64, r * 128, bh);
-      long long tw0 = clock64();
-      // wait for our own copies before the CTA may retire (bounded)
-      while (!(mbar_try_wait(&bar->c_full, 0) && mbar_try_wait(&bar->q_full, 0)) &&
-             clock64() - tw0 < kWaitLimitCycles) {
+      if (!ok || *abort_flag) {
+        // let every copy started here land before the CTA retires (bounded)
+        long long tw0 = clock64();
+        while (loads > 0 && !mbar_try_wait(&bar->c_full, (loads - 1) & 1) &&
+               clock64() - tw0 < kWaitLimitCycles) {
+        }
+        for (int it = (q_issued > 2 ? q_issued - 2 : 0); it < q_issued; ++it) {
+          tw0 = clock64();
+          while (!mbar_try_wait(&bar->q_full[it & 1], (it >> 1) & 1) &&
+                 clock64() - tw0 < kWaitLimitCycles) {
+          }
+        }
       }
     }
   } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane_id() == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, p.C, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      bool ok = mbar_wait(&bar->c_full, 0, abort_flag, p.status) &&
-                mbar_wait(&bar->q_full, 0, abort_flag, p.status);
-      if (ok) {
+      int cur = -1, loads = 0;
+      bool ok = true;
+      for (int it = 0; it < n && ok; ++it) {
+        const int u = T0 + it, bh = u / p.nqb;
+        const int b = it & 1;
+        if (bh != cur) {
+          ok = mbar_wait(&bar->c_full, loads & 1, abort_flag, p.status);
+          ++loads;
+          cur = bh;
+          if (!ok) break;
+        }
+        if (!mbar_wait(&bar->q_full[b], (it >> 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
+        // S(it) follows O(it-1) in the pipe, which has read P(it-1) from the same columns
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t o = (kk & 3) * 32;
-          mma_bf16_ss(tmem + Cf::kColS, sdesc_sw128(q_addr + (kk >> 2) * Cf::kQPanel + o, 16, 1024),
+          mma_bf16_ss(tmem + Cf::kColS,
+                      sdesc_sw128(q_addr + b * Cf::kQBytes + (kk >> 2) * Cf::kQPanel + o, 16, 1024),
                       sdesc_sw128(k_addr + (kk >> 2) * Cf::kCPanel + o, 16, 1024), idesc_s,
                       kk > 0 ? 1u : 0u);
         }
         tc_commit(&bar->s_full);
-        ok = mbar_wait(&bar->p_full, 0, abort_flag, p.status);
-      }
-      if (ok) {
+        tc_commit(&bar->q_empty[b]);
+        if (!mbar_wait(&bar->p_full, it & 1, abort_flag, p.status)) break;
+        // the merge of tile it-1 has read O
+        if (it > 0 && !mbar_wait(&bar->o_empty, (it - 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         for (int kk = 0; kk < p.C / 16; ++kk)
           mma_bf16_ts(tmem + Cf::kColO, tmem + Cf::kColS + kk * 8,
                       sdesc_sw128(v_addr + kk * 16 * 128, Cf::kCPanel, 1024), idesc_o,
                       kk > 0 ? 1u : 0u);
         tc_commit(&bar->o_full);
+        if (it + 1 < n && (u + 1) / p.nqb != bh) tc_commit(&bar->kv_free);
       }
       if (*abort_flag) {
         tc_commit(&bar->drain);
@@ -1139,83 +1208,153 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
       }
     }
   } else {
+    // ------------------------------------------------------------ softmax / merge
     // Every tcgen05.ld / st below is warp-collective: the branches around them
     // are warp-uniform, and only the global loads and stores depend on the row.
+    // The four warps leave the tile loop together (a barrier that ORs their
+    // failures), so none is left at a named barrier. Per tile: P from S, then
+    // (while the tensor core forms O) the row's sparse output is fetched and
+    // the next tile's biases are built, then the merge.
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&bar->s_full, 0, abort_flag, p.status));
-    float m = -INFINITY, den = 0.0f;
-    if (ok) {
-      tc_fence_after();
-      for (int ch = 0; ch < p.C / 32; ++ch) {
-        uint32_t s[32];
-        tmem_ld_32x32b_x32(lane_base + Cf::kColS + ch * 32, s);
-        tmem_ld_wait();
-        reg_fence(s);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          m = fmaxf(m, fmaf(u2f(s[i]), p.scale_log2, sBias[ch * 32 + i]));
+    const int tw = (p.nkb + 31) / 32;
+    // biases of tile it into sBias[it % 2]: bias_b = log2 of cluster b's keys
+    // outside the tile's computed key tiles (the bitmap of its CSR row)
+    auto build_bias = [&](int it) {
+      const int u = T0 + it, bh = u / p.nqb, r = u - bh * p.nqb;
+      for (int i = tid; i < tw; i += 128) bar->tiles[i] = 0u;
+      named_bar_sync(1, 128);
+      const int row = bh * p.nqb + r;
+      const int c0 = p.row_ptr[row], c1 = p.row_ptr[row + 1];
+      for (int i = c0 + tid; i < c1; i += 128) {
+        const int t = p.col_idx[i];
+        if (t >= 0 && t < p.nkb) atomicOr(&bar->tiles[t >> 5], 1u << (t & 31));
+        else atomicOr(p.status, kDevErrBounds);
       }
-      if (p.C % 32 != 0) {
-        uint32_t s[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
-              "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]),
-              "=r"(s[12]), "=r"(s[13]), "=r"(s[14]), "=r"(s[15])
-            : "r"(lane_base + Cf::kColS + (p.C / 32) * 32)
-            : "memory");
-        tmem_ld_wait();
-        reg_fence(s);
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          m = fmaxf(m, fmaf(u2f(s[i]), p.scale_log2, sBias[(p.C / 32) * 32 + i]));
-      }
-      const float mu = m == -INFINITY ? 0.0f : m;
-      // P in 16-column chunks: S columns [16 ch, 16 ch + 16) -> P columns [8 ch, 8 ch + 8)
-      for (int ch = 0; ch < p.C / 16; ++ch) {
-        uint32_t s[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
-              "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]),
-              "=r"(s[12]), "=r"(s[13]), "=r"(s[14]), "=r"(s[15])
-            : "r"(lane_base + Cf::kColS + ch * 16)
-            : "memory");
-        tmem_ld_wait();
-        reg_fence(s);
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int b = ch * 16 + 2 * i;
-          const float p0 = fast_exp2(fmaf(u2f(s[2 * i]), p.scale_log2, sBias[b]) - mu);
-          const float p1 = fast_exp2(fmaf(u2f(s[2 * i + 1]), p.scale_log2, sBias[b + 1]) - mu);
-          den += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+      named_bar_sync(1, 128);
+      const int32_t* off = p.offsets_k + static_cast<size_t>(bh) * (p.C + 1);
+      float* bias = sBias + (it & 1) * kMaxC;
+      for (int b = tid; b < p.C; b += 128) {
+        const int k0 = off[b], k1 = off[b + 1];
+        int covered = 0;
+        if (k1 > k0) {
+          for (int t = k0 / p.bk; t <= (k1 - 1) / p.bk; ++t) {
+            if ((bar->tiles[t >> 5] >> (t & 31)) & 1u) {
+              const int lo = max(k0, t * p.bk), hi = min(k1, (t + 1) * p.bk);
+              covered += hi - lo;
+            }
+          }
         }
-        // P of these 16 clusters overwrites S columns the loop has already read
-        tmem_st_32x32b_x8(lane_base + Cf::kColS + ch * 8, pk);
+        const int nb = k1 - k0 - covered;
+        bias[b] = nb > 0 ? __log2f(static_cast<float>(nb)) : -INFINITY;
       }
-      tmem_st_wait();
-    }
-    tc_fence_before();
-    mbar_arrive(&bar->p_full);
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->o_full, 0, abort_flag, p.status));
-    tc_fence_after();
-    // merge with the sparse output of this row (rows past N only take part in
-    // the warp's tensor-memory loads)
-    const int qrow = r * 128 + tid;
-    const bool row_ok = qrow < p.N;
-    if (ok) {
+      named_bar_sync(1, 128);  // the biases are complete, and the bitmap may be rebuilt
+    };
+    bool ok = true;
+    if (n > 0) build_bias(0);
+    for (int it = 0; it < n; ++it) {
+      if (named_bar_or(1, 128, !ok || *abort_flag != 0)) break;
+      const int u = T0 + it, bh = u / p.nqb, r = u - bh * p.nqb;
+      const float* bias = sBias + (it & 1) * kMaxC;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar->s_full, it & 1, abort_flag, p.status));
+      float m = -INFINITY, den = 0.0f;
+      if (ok) {
+        tc_fence_after();
+        // S in 32-column chunks, two loads in flight per wait; the C % 32 = 16
+        // tail alone
+        const int n32 = p.C / 32;
+        const float* tail_bias = bias + n32 * 32;
+        for (int ch = 0; ch < n32; ch += 2) {
+          uint32_t sa[32], sb[32];
+          const bool two = ch + 1 < n32;  // warp-uniform
+          tmem_ld_32x32b_x32(lane_base + Cf::kColS + ch * 32, sa);
+          if (two) tmem_ld_32x32b_x32(lane_base + Cf::kColS + (ch + 1) * 32, sb);
+          tmem_ld_wait();
+          reg_fence(sa);
+          reg_fence(sb);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) m = fmaxf(m, fmaf(u2f(sa[i]), p.scale_log2, bias[ch * 32 + i]));
+          if (two) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              m = fmaxf(m, fmaf(u2f(sb[i]), p.scale_log2, bias[(ch + 1) * 32 + i]));
+          }
+        }
+        if (p.C % 32 != 0) {
+          uint32_t s[16];
+          tmem_ld_32x32b_x16(lane_base + Cf::kColS + n32 * 32, s);
+          tmem_ld_wait();
+          reg_fence(s);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) m = fmaxf(m, fmaf(u2f(s[i]), p.scale_log2, tail_bias[i]));
+        }
+        const float mu = m == -INFINITY ? 0.0f : m;
+        // P: S columns [32 ch, 32 ch + 32) -> P columns [16 ch, 16 ch + 16), which
+        // hold S columns already read
+        auto exp_chunk = [&](const uint32_t (&s)[32], int ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int b = ch * 32 + 2 * i;
+            const float p0 = fast_exp2(fmaf(u2f(s[2 * i]), p.scale_log2, bias[b]) - mu);
+            const float p1 = fast_exp2(fmaf(u2f(s[2 * i + 1]), p.scale_log2, bias[b + 1]) - mu);
+            den += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_32x32b_x16(lane_base + Cf::kColS + ch * 16, pk);
+        };
+        for (int ch = 0; ch < n32; ch += 2) {
+          uint32_t sa[32], sb[32];
+          const bool two = ch + 1 < n32;  // warp-uniform
+          tmem_ld_32x32b_x32(lane_base + Cf::kColS + ch * 32, sa);
+          if (two) tmem_ld_32x32b_x32(lane_base + Cf::kColS + (ch + 1) * 32, sb);
+          tmem_ld_wait();
+          reg_fence(sa);
+          reg_fence(sb);
+          exp_chunk(sa, ch);
+          if (two) exp_chunk(sb, ch + 1);
+        }
+        if (p.C % 32 != 0) {
+          uint32_t s[16];
+          tmem_ld_32x32b_x16(lane_base + Cf::kColS + n32 * 32, s);
+          tmem_ld_wait();
+          reg_fence(s);
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float p0 = fast_exp2(fmaf(u2f(s[2 * i]), p.scale_log2, tail_bias[2 * i]) - mu);
+            const float p1 =
+                fast_exp2(fmaf(u2f(s[2 * i + 1]), p.scale_log2, tail_bias[2 * i + 1]) - mu);
+            den += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_32x32b_x8(lane_base + Cf::kColS + n32 * 16, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar->p_full);
+      }
+      // this row's sparse output and log-sum-exp, fetched while O is formed
+      // (rows past N only take part in the warp's tensor-memory loads)
+      const int qrow = r * 128 + tid;
+      const bool row_ok = qrow < p.N;
       const size_t ro = static_cast<size_t>(bh) * p.N + (row_ok ? qrow : 0);
-      const float lse2 = row_ok ? p.lse[ro] * 1.4426950408889634f : -INFINITY;
+      uint4* dst = reinterpret_cast<uint4*>(p.os + ro * D);
+      uint4 sp[D / 8];
+      float lse2 = -INFINITY;
+      if (ok && row_ok) {
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) sp[i] = dst[i];
+        lse2 = p.lse[ro] * 1.4426950408889634f;
+      }
+      if (it + 1 < n) build_bias(it + 1);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->o_full, it & 1, abort_flag, p.status));
+      if (!ok) continue;  // leaves at the next iteration's barrier
+      tc_fence_after();
       const float M = fmaxf(lse2, m);
       const float a = lse2 == -INFINITY ? 0.0f : fast_exp2(lse2 - M);
       const float c = m == -INFINITY ? 0.0f : fast_exp2(m - M);
       const float tot = a + den * c;
       const float inv = tot > 0.0f ? 1.0f / tot : 0.0f;  // no key at all: O = 0
-      svg_bf16* orow = p.os + ro * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
@@ -1223,11 +1362,10 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
         tmem_ld_wait();
         reg_fence(o);
         if (!row_ok) continue;
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
         uint32_t pk[16];
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
-          const uint4 in = dst[v4];
+          const uint4 in = sp[ch * 4 + v4];
           const uint32_t w[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -1239,11 +1377,12 @@ __global__ void __launch_bounds__(kEarThreads, 1) ear_compensate_kernel(const __
         }
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4)
-          dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          dst[ch * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
       }
-    } else if (!ok && tid == 0) {
-      atomicOr(p.status, kDevErrTimeout);
+      tc_fence_before();
+      mbar_arrive(&bar->o_empty);
     }
+    if (!ok && tid == 0) atomicOr(p.status, kDevErrTimeout);
   }
 
   tc_fence_before();
@@ -1355,7 +1494,7 @@ cudaError_t launch_cluster_sort(int32_t BH, int32_t N, int32_t C, const int32_t*
 
 cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, const svg_bf16* x,
                                  const int32_t* order, const int32_t* offsets, const float* c_in,
-                                 float* c_out, void* ws, cudaStream_t stream) {
+                                 float* c_out, void* ws, int* status, cudaStream_t stream) {
   const KWs w = carve(ws, BH, N, D, C);
   const int nchunks = (N + kChunkRows - 1) / kChunkRows;
   const dim3 g_sum(static_cast<unsigned>((nchunks + kChunkWarps - 1) / kChunkWarps),
@@ -1368,7 +1507,7 @@ cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, co
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ChunkCfg<128>::kSmem);
     if (e != cudaSuccess) return e;
     kmeans_chunk_sum_kernel<128><<<g_sum, 32 * kChunkWarps, ChunkCfg<128>::kSmem, stream>>>(
-        x, order, offsets, N, C, nchunks, w.partial);
+        x, order, offsets, N, C, nchunks, w.partial, status);
     kmeans_mean_kernel<128><<<g_mean, 32 * kChunkWarps, 0, stream>>>(w.partial, offsets, C,
                                                                      nchunks, c_in, c_out);
   } else {
@@ -1376,7 +1515,7 @@ cudaError_t launch_kmeans_update(int32_t BH, int32_t N, int32_t D, int32_t C, co
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ChunkCfg<64>::kSmem);
     if (e != cudaSuccess) return e;
     kmeans_chunk_sum_kernel<64><<<g_sum, 32 * kChunkWarps, ChunkCfg<64>::kSmem, stream>>>(
-        x, order, offsets, N, C, nchunks, w.partial);
+        x, order, offsets, N, C, nchunks, w.partial, status);
     kmeans_mean_kernel<64><<<g_mean, 32 * kChunkWarps, 0, stream>>>(w.partial, offsets, C, nchunks,
                                                                     c_in, c_out);
   }
@@ -1408,7 +1547,7 @@ cudaError_t launch_kmeans(int32_t BH, int32_t N, int32_t D, int32_t C, int32_t i
         cudaSuccess)
       return e;
     if ((e = launch_kmeans_update(BH, N, D, C, x, order, offsets, bufs[cur], bufs[cur ^ 1], ws,
-                                  stream)) != cudaSuccess)
+                                  status, stream)) != cudaSuccess)
       return e;
     cur ^= 1;
   }
@@ -1521,21 +1660,29 @@ cudaError_t launch_ear_compensate(int32_t BH, int32_t N, int32_t D, int32_t C, i
   p.N = N;
   p.C = C;
   p.bk = bk;
+  p.BH = BH;
   p.nqb = (N + 127) / 128;
   p.nkb = (N + bk - 1) / bk;
   p.scale_log2 = scale * 1.4426950408889634f;
+  // persistent: one CTA per SM (each takes all tensor-memory columns)
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const long long tiles = static_cast<long long>(BH) * p.nqb;
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
   if (D == 128) {
     auto kern = ear_compensate_kernel<128>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   EarCfg<128>::kSmem)) != cudaSuccess)
       return e;
-    kern<<<dim3(p.nqb, BH), kEarThreads, EarCfg<128>::kSmem, stream>>>(p);
+    kern<<<grid, kEarThreads, EarCfg<128>::kSmem, stream>>>(p);
   } else {
     auto kern = ear_compensate_kernel<64>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   EarCfg<64>::kSmem)) != cudaSuccess)
       return e;
-    kern<<<dim3(p.nqb, BH), kEarThreads, EarCfg<64>::kSmem, stream>>>(p);
+    kern<<<grid, kEarThreads, EarCfg<64>::kSmem, stream>>>(p);
   }
   return cudaGetLastError();
 }
