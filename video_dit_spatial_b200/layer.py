@@ -232,8 +232,13 @@ class SemanticSparseLayer:
         self.scale = float(d ** -0.5 if scale is None else scale)
         dev = self.device = torch.device(device)
         BH = self.BH
-        ws = max(svg2_kmeans_workspace_bytes(BH, N, d, Cq), svg2_kmeans_workspace_bytes(BH, N, d, Ck))
-        self.workspace = torch.empty(ws // 4 + 64, dtype=torch.float32, device=dev)
+        # the query and key clusterings run side by side on two streams, each
+        # with its own workspace
+        self.workspace = torch.empty(svg2_kmeans_workspace_bytes(BH, N, d, Cq) // 4 + 64,
+                                     dtype=torch.float32, device=dev)
+        self.workspace_k = torch.empty(svg2_kmeans_workspace_bytes(BH, N, d, Ck) // 4 + 64,
+                                       dtype=torch.float32, device=dev)
+        self._side = torch.cuda.Stream(device=dev)
         i32 = dict(dtype=torch.int32, device=dev)
         self.cq = torch.empty((BH, Cq, d), dtype=torch.float32, device=dev)
         self.ck = torch.empty((BH, Ck, d), dtype=torch.float32, device=dev)
@@ -267,22 +272,30 @@ class SemanticSparseLayer:
         self._v = v
         from . import svg2_build_tile_csr, svg2_kmeans, svg2_select_clusters
         BH, N, d = self.BH, self.N, self.d
+        main = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if isinstance(main, int):
+            main = torch.cuda.ExternalStream(main, device=self.device)
+        # keys (and the value statistics) on the side stream, joined before the
+        # selection; both start after what `main` holds so far (q, k, v written)
+        side = self._side
+        side.wait_stream(main)
         svg2_kmeans(BH, N, d, self.Cq, self.iters, q, self.cq, self.assign_q, self.order_q,
-                    self.offsets_q, self.workspace, stream=stream)
+                    self.offsets_q, self.workspace, stream=main)
         svg2_kmeans(BH, N, d, self.Ck, self.iters, k, self.ck, self.assign_k, self.order_k,
-                    self.offsets_k, self.workspace, stream=stream)
+                    self.offsets_k, self.workspace_k, stream=side)
         disp = None
         if self.ear_tau is not None:
             from . import svg2_cluster_value_stats
             svg2_cluster_value_stats(BH, N, d, self.Ck, self._v, self.order_k, self.offsets_k,
-                                     self.vbar, self.disp, stream=stream)
+                                     self.vbar, self.disp, stream=side)
             disp = self.disp
+        main.wait_stream(side)
         svg2_select_clusters(BH, d, self.Cq, self.Ck, self.scale, self.top_p, self.cq, self.ck,
                              self.offsets_k, self.sel, disp=disp, tau=self.ear_tau or 0.0,
-                             stream=stream)
+                             stream=main)
         svg2_build_tile_csr(BH, N, self.Cq, self.Ck, self.block_q, self.block_k, self.offsets_q,
                             self.offsets_k, self.sel, self.row_ptr, self.col_idx, self.counts,
-                            stream=stream)
+                            stream=main)
 
     def attend(self, q, k, v, o, lse=None, stream=None) -> None:
         """Permute, block-sparse attention over the planned tiles, un-permute."""
