@@ -369,13 +369,16 @@ def _unpack_sel(sel, Ck):
             .reshape(bits.shape[0], bits.shape[1], -1)[..., :Ck].astype(bool))
 
 
+@pytest.mark.parametrize("wname", ["hunyuan_B1_H24_d128_T33_P3600_L256",
+                                   "cogvideox15_B1_H48_d64_T11_P4080_L226"],
+                         ids=["hunyuan_d128", "cogvideox_d64"])
 @pytest.mark.parametrize("ear_tau", [None, 0.01], ids=["svg2", "ear"])
-def test_semantic_layer_full_size_sampled_rows(svg, ear_tau):
-    """HunyuanVideo-shaped length (N = 119 056, d = 128), 2 heads of the seeded
-    layer, C = 256 clusters, 10 iterations, top-p 0.9, with and without SVG-EAR
-    routing: every part of the plan the GPU builds is checked against what
-    defines it, and the output against the oracle's attention over that plan
-    on sampled rows.
+def test_semantic_layer_full_size_sampled_rows(svg, ear_tau, wname):
+    """Full-length workloads (HunyuanVideo-shaped N = 119 056, d = 128, and
+    CogVideoX-shaped N = 45 106, d = 64), 2 heads of the seeded layer, C = 256
+    clusters, 10 iterations, top-p 0.9, with and without SVG-EAR routing: every
+    part of the plan the GPU builds is checked against what defines it, and the
+    output against the oracle's attention over that plan on sampled rows.
       - order and offsets: the stable cluster order of the GPU's own assignment;
       - selection: each query cluster's kept set is a valid top-p prefix of the
         oracle's weights from the GPU's centroids (with routing: every cluster
@@ -387,7 +390,7 @@ def test_semantic_layer_full_size_sampled_rows(svg, ear_tau):
       - output: element-wise within the attention bars on sampled rows."""
     import svg_inputs as SI
     from video_dit_spatial_b200.layer import SemanticSparseLayer
-    wl = SI.HUNYUAN.replace(H=2, n_spatial=1)
+    wl = SI.WORKLOADS[wname].replace(H=2, n_spatial=1)
     q, k, v = SI.make_qkv(wl)
     B, H, N, d, C, top_p = 1, 2, wl.N, wl.d, 256, 0.9
     layer = SemanticSparseLayer(B, H, N, d, Cq=C, Ck=C, iters=10, top_p=top_p, ear_tau=ear_tau)
@@ -457,7 +460,8 @@ def test_semantic_layer_full_size_sampled_rows(svg, ear_tau):
             want = S2.ear_attention_rows(qn, kn, vn, oq_, ok_, offk, ck, vbar, bm, 128, 128,
                                          scale, rows)
         density = float(np.diff(rp[h * nqb:(h + 1) * nqb + 1]).sum()) / (nqb * layer.nkb)
-        print(f"SVG2-FULL {'ear' if ear_tau else 'svg2'} head {h}: tile density {density:.3f}, "
+        label = f"{'ear' if ear_tau else 'svg2'} d{d} head {h}"
+        print(f"SVG2-FULL {label}: tile density {density:.3f}, "
               f"{len(tiles)} tiles and {len(rows)} rows checked")
-        assert_close(got[0, h][rows], want, f"SVG2 full size {'ear' if ear_tau else 'svg2'} head {h}")
+        assert_close(got[0, h][rows], want, f"SVG2 full size {label}")
     status_clean()
