@@ -198,3 +198,59 @@ def test_ear_layer_end_to_end_on_planted_frames(svg):
                                      np.arange(N))
         assert_close(got[0, h], want, f"EAR layer head {h}")
     status_clean()
+
+
+def test_ear_compensation_many_short_heads(svg):
+    """96 heads of 3 query tiles each (288 tiles over at most one CTA per SM):
+    the persistent compensation kernel moves between heads inside most CTAs,
+    reloading the centroids each time; sampled rows of every head against the
+    oracle."""
+    BH, N, d, Ck, Cq, bk, scale = 96, 300, 64, 16, 4, 128, 1.0 / 8.0
+    rng = np.random.default_rng(96)
+    q, k, v = (rand_bf16((BH, N, d), seed=960 + i) for i in range(3))
+    plans = _plans(rng, BH, N, Cq, Ck, 0.3)
+    qn, kn, vn = to_f64(q), to_f64(k), to_f64(v)
+    kbar = np.zeros((BH, Ck, d))
+    vbar = np.zeros((BH, Ck, d))
+    for h in range(BH):
+        ok_, offk = plans[h][2], plans[h][3]
+        for b in range(Ck):
+            mem = ok_[offk[b]:offk[b + 1]]
+            if mem.size:
+                kbar[h, b] = kn[h, mem].mean(axis=0)
+        vbar[h] = S2.cluster_value_stats(vn[h], ok_, offk)[0]
+    order_q = _dev_i32(np.stack([p[0] for p in plans]))
+    offs_q = _dev_i32(np.stack([p[1] for p in plans]))
+    order_k = _dev_i32(np.stack([p[2] for p in plans]))
+    offs_k = _dev_i32(np.stack([p[3] for p in plans]))
+    nqb, nkb = -(-N // 128), -(-N // bk)
+    row_ptr = torch.empty(BH * nqb + 1, dtype=torch.int32, device="cuda")
+    col_idx = torch.empty(BH * nqb * nkb, dtype=torch.int32, device="cuda")
+    counts = torch.empty(BH * nqb, dtype=torch.int32, device="cuda")
+    svg.svg2_build_tile_csr(BH, N, Cq, Ck, 128, bk, offs_q, offs_k,
+                            _pack([p[4] for p in plans], Ck), row_ptr, col_idx, counts)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    qs, ks, vs, os_, o = (torch.empty_like(qd) for _ in range(5))
+    lse = torch.empty((BH, N), device="cuda")
+    svg.svg2_gather_rows(BH, N, d, qd, order_q, qs)
+    svg.svg2_gather_rows(BH, N, d, kd, order_k, ks)
+    svg.svg2_gather_rows(BH, N, d, vd, order_k, vs)
+    svg.svg2_sparse_attention(BH, N, d, bk, scale, qs, ks, vs, row_ptr, col_idx, os_, lse)
+    ws = torch.empty(svg.svg2_ear_workspace_bytes(BH, d, Ck) // 4 + 64, device="cuda")
+    svg.svg2_ear_compensate(BH, N, d, Ck, bk, scale, qs,
+                            torch.from_numpy(kbar.astype(np.float32)).cuda(),
+                            torch.from_numpy(vbar.astype(np.float32)).cuda(), offs_k, row_ptr,
+                            col_idx, os_, lse, ws)
+    svg.svg2_scatter_rows(BH, N, d, os_, order_q, o)
+    torch.cuda.synchronize()
+    got = to_f64(o)
+    for h in range(BH):
+        oq_, offq, ok_, offk, sel = plans[h]
+        bm = S2.semantic_block_mask(offq, offk, sel, 128, bk)
+        rows = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 10, replace=False)]))
+        want = S2.ear_attention_rows(qn[h], kn[h], vn[h], oq_, ok_, offk,
+                                     kbar[h].astype(np.float32).astype(np.float64),
+                                     vbar[h].astype(np.float32).astype(np.float64), bm, 128, bk,
+                                     scale, rows)
+        assert_close(got[h][rows], want, f"EAR many heads head {h}")
+    status_clean()
