@@ -59,8 +59,10 @@ def _check_assignment(x, cent, got):
 
 
 # BH, N, d, C, planted
+# the last case has more heads than SMs (one assignment CTA per head) and
+# chunks shorter than one 256-row chunk per head
 STEP_CASES = [(2, 1000, 64, 16, False), (2, 1500, 128, 48, False), (1, 3000, 128, 256, True),
-              (3, 777, 128, 32, True)]
+              (3, 777, 128, 32, True), (160, 200, 64, 16, True)]
 
 
 @pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: "BH{}N{}d{}C{}".format(*c[:4]))
